@@ -1,0 +1,421 @@
+"""Benchmark of the block-sparse spatio-temporal attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload spatial_75600|temporal_75600|mixed_75600|p1440_302400]
+                    [--bq 128 --bk 128] [--mode split|naive] [--no-extras]
+
+A step is one call of svg_attention_fwd (split mode: full tiles unmasked, boundary tiles
+masked) over the whole workload, Q/K/V/O resident in HBM (774 MB at 75,600 tokens, larger
+than the 126 MB L2, so no flush is needed between steps). Tile maps are built once per
+geometry (the design caches them) and timed separately, as are the token permutation, the
+dense baseline, the naive and the rounded modes. Multi-GPU runs are independent replicas
+(the path has no exchange step): every rank runs the same workload; the step time is the
+max over ranks and `value` sums the work of all ranks.
+
+Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle instead (rank 0
+only, bounded row sample per step, full-call time extrapolated by rows).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_spatio_flash_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "ms/call & effective TFLOP/s, 75,600-tok 10-head d128 bf16 sparse attention"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+def time_events(fn, iters, stream):
+    """Mean ms per call over `iters` calls, CUDA events on the launching stream."""
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for _ in range(iters):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def workload_flops(w, summaries):
+    """(effective, visited, executed) FLOP per call: 4*d*pairs; retained / in-range visited area /
+    MMA work actually issued (128-row halves x bk key tiles)."""
+    eff = vis = exe = 0
+    for r in w.routes:
+        s = summaries[r]
+        eff += 4 * w.d * s.retained_map
+        vis += 4 * w.d * s.visited_area
+        exe += 4 * w.d * s.pair_half_tiles * 128 * w.bk
+    return eff, vis, exe
+
+
+def oracle_sample(w, q, k, v, rows_per_head):
+    """Time the fp64 oracle on a seeded row sample of every head; return (seconds, rows, threads)."""
+    import oracle
+    t0 = time.perf_counter()
+    nrows = 0
+    for h in range(w.heads):
+        rows = syn.sample_rows(w.replace(sample_rows=rows_per_head), h).numpy()
+        rows = rows[:rows_per_head]
+        oracle.attention_rows(q[h], k[h], v[h], rows, route=w.routes[h], layout=w.layout, T=w.frames,
+                              S=w.frame_size, frame_window=w.frame_window, band=w.spatial_band, F0=w.sink_frames)
+        nrows += len(rows)
+    return time.perf_counter() - t0, nrows, oracle.num_threads()
+
+
+def closed_form_effective_flops(w):
+    """4*d*retained for the exact masks, from the oracle's closed-form-pinned brute force is
+    too slow here; the tile-map summary gives the same number on the GPU path. For the CPU
+    arm the retained count is computed by the oracle once (exact)."""
+    import oracle
+    tot = 0
+    for r in set(w.routes):
+        n = oracle.retained_pairs(r, w.frames, w.frame_size, w.frame_window, w.spatial_band, w.sink_frames)
+        tot += n * sum(1 for x in w.routes if x == r)
+    return 4 * w.d * tot
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return 0
+    q, k, v = syn.make_qkv(w)
+    eff = closed_form_effective_flops(w)
+    rows = args.ref_rows
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_sample(w, q, k, v, max(4, rows // 8))
+    times = []
+    nthreads = 1
+    for _ in range(args.steps):
+        sec, nrows, nthreads = oracle_sample(w, q, k, v, rows)
+        times.append(sec * (w.tokens * w.heads) / nrows)  # extrapolated full-call seconds
+    t = statistics.mean(times)
+    value = eff / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{rows} seeded query rows per head x {w.heads} heads per step; full-call time "
+                                   f"extrapolated linearly by rows"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=syn.SPATIAL_75K.name)
+    ap.add_argument("--bq", type=int, default=128)
+    ap.add_argument("--bk", type=int, default=128)
+    ap.add_argument("--mode", default="split", choices=["split", "naive"])
+    ap.add_argument("--no-extras", action="store_true", help="skip the side measurements")
+    ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=48, help="oracle rows per head per --impl reference step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_env()
+    w = syn.WORKLOADS[args.workload].replace(bq=args.bq, bk=args.bk)
+
+    if args.impl == "reference":
+        return run_reference(args, w, world, rank)
+
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    from block_sparse_spatio_flash_b200 import svg as S
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    P, peak_kind = peaks()
+    g = S.make_geom(w.frames, w.grid_h, w.grid_w)
+    m = S.make_mask(w.frame_window, w.spatial_band, w.sink_frames, w.variant, w.layout)
+    t = S.make_tile(w.bq, w.bk)
+    routes = list(w.routes)
+    mode = S.SVG_MODE_SPLIT if args.mode == "split" else S.SVG_MODE_NAIVE
+
+    q_cpu, k_cpu, v_cpu = syn.make_qkv(w)
+    q, k, v = (x.to(dev) for x in (q_cpu, k_cpu, v_cpu))
+    if any(routes):  # temporal heads run in their own token order (permutation timed separately)
+        qp, kp, vp = (torch.empty_like(x) for x in (q, k, v))
+        for a, b_ in ((q, qp), (k, kp), (v, vp)):
+            S.svg_permute(a, b_, routes, g, m)
+    else:
+        qp, kp, vp = q, k, v
+    o = torch.empty_like(qp)
+    scratch = S.alloc_scratch(dev)
+
+    ws = [None, None]
+    summ = [None, None]
+    for c in sorted(set(routes)):
+        ws[c] = S.alloc_workspace(g, t, dev)
+        S.svg_build_tilemap(g, m, t, c, ws[c])
+        summ[c] = S.svg_tilemap_summary(ws[c])
+    eff_flop, vis_flop, exe_flop = workload_flops(w, summ)
+
+    def step():
+        S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, mode=mode, scratch=scratch)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = S.svg_read_status(scratch)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {S.svg_error_string(status)}")
+
+    # ---------------------------------------------------------------- timed region
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms = total_ms / args.steps
+    status = S.svg_read_status(scratch)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {S.svg_error_string(status)}")
+    value = world * eff_flop / (ms * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    # ---------------------------------------------------------------- roofline of the attention kernel
+    peak = float(P["bf16_tflops"])
+    achieved = vis_flop / (statistics.mean(per_step) * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "attn_kernel<128,128> (split)", "flop_definition": "4*d*(in-range area of visited tiles)",
+                "peak_kind": f"{peak_kind} bf16 burst"}
+
+    extras = {}
+    if not args.no_extras:
+        extras = side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws, summ, P, stream,
+                                   dev)
+
+    # ---------------------------------------------------------------- end to end through host buffers
+    e2e = end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream,
+                     args)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        sec, nrows, nthreads = oracle_sample(w, q_cpu, k_cpu, v_cpu, args.cpu_rows)
+        full = sec * (w.tokens * w.heads) / nrows
+        cpu = {"value": eff_flop / full / 1e12, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
+               "sample": f"{args.cpu_rows} seeded query rows per head x {w.heads} heads ({nrows} rows, "
+                         f"{sec:.1f} s); full-call time extrapolated linearly by rows = {full:.1f} s",
+               "ms_per_call_extrapolated": full * 1e3}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d,
+                       "routes": "".join("S" if r == 0 else "T" for r in routes),
+                       "frame_window": w.frame_window, "spatial_band": w.spatial_band, "sink_frames": w.sink_frames,
+                       "bq": w.bq, "bk": w.bk, "mode": args.mode, "parallelism": f"replicas x{world}",
+                       "l2": "no flush: Q/K/V/O = %.0f MB > 126 MB L2" % (4 * w.heads * w.tokens * w.d * 2 / 1e6)},
+            "ms_per_call": ms,
+            "effective_flop_per_call": eff_flop, "visited_flop_per_call": vis_flop, "executed_flop_per_call": exe_flop,
+            "visited_tflops": vis_flop / (ms * 1e-3) / 1e12,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clocks, "extras": extras,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws, summ, P, stream, dev):
+    out = {}
+    iters = 10
+    hbm = float(P["hbm_gbs"])
+    # tile-map build (integer, once per geometry)
+    ms = time_events(lambda: [S.svg_build_tilemap(g, m, t, c, ws[c]) for c in sorted(set(routes))], 5, stream)
+    out["tilemap_build_ms"] = ms
+    # permutation, one [H, N, d] tensor (temporal heads reordered, spatial heads copied)
+    tmp = torch.empty_like(q)
+    ms = time_events(lambda: S.svg_permute(q, tmp, routes, g, m), iters, stream)
+    nbytes = 2 * q.numel() * 2
+    out["permute_ms_per_tensor"] = ms
+    out["permute_gbs"] = nbytes / (ms * 1e-3) / 1e9
+    out["permute_hbm_frac"] = out["permute_gbs"] / hbm
+    # dense baseline (same kernel, every tile full)
+    ms = time_events(lambda: S.svg_dense_attention_fwd(qp, kp, vp, o, bk=t.bk, scratch=scratch), 3, stream)
+    dense_flop = 4 * w.d * w.tokens * w.tokens * w.heads
+    out["dense_ms"] = ms
+    out["dense_tflops"] = dense_flop / (ms * 1e-3) / 1e12
+    # naive mode (every visited tile masked)
+    ms = time_events(lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t,
+                                                 mode=S.SVG_MODE_NAIVE, scratch=scratch), 5, stream)
+    out["naive_ms"] = ms
+    # split mode again for the ratio
+    ms_split = time_events(lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t,
+                                                       mode=S.SVG_MODE_SPLIT, scratch=scratch), 5, stream)
+    out["split_ms"] = ms_split
+    out["split_vs_dense"] = out["dense_ms"] / ms_split
+    # rounded (tile-aligned) masks
+    mr = S.make_mask(w.frame_window, w.spatial_band, w.sink_frames, S.SVG_MASK_ROUNDED, w.layout)
+    wr = [None, None]
+    rs = {}
+    for c in sorted(set(routes)):
+        wr[c] = S.alloc_workspace(g, t, dev)
+        S.svg_build_tilemap(g, mr, t, c, wr[c])
+        rs[c] = S.svg_tilemap_summary(wr[c])
+    ms = time_events(lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, wr[0], wr[1], g, mr, t, scratch=scratch),
+                     5, stream)
+    out["rounded_ms"] = ms
+    for name, sm in (("exact", summ), ("rounded", rs)):
+        tot_tiles = sum(sm[c].n_full + sm[c].n_boundary + sm[c].n_empty for c in sorted(set(routes)))
+        vis = sum(sm[c].n_full + sm[c].n_boundary for c in sorted(set(routes)))
+        bnd = sum(sm[c].n_boundary for c in sorted(set(routes)))
+        kept = sum(sm[c].retained_map * sum(1 for r in routes if r == c) for c in sorted(set(routes)))
+        out[f"{name}_boundary_frac_of_visited"] = bnd / max(vis, 1)
+        out[f"{name}_visited_frac_of_all"] = vis / max(tot_tiles, 1)
+        out[f"{name}_retained_frac"] = kept / (w.heads * w.tokens ** 2)
+    st = S.svg_read_status(scratch)
+    out["status"] = st
+    return out
+
+
+def end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream, args):
+    """Same metric through the public API with host buffers: pinned H2D of Q/K/V, permutation of
+    temporal heads, attention, inverse permutation, D2H of O -- all inside the timed region."""
+    qh, kh, vh = (x.pin_memory() for x in (q_cpu, k_cpu, v_cpu))
+    oh = torch.empty_like(q_cpu).pin_memory()
+    qd, kd, vd = (torch.empty_like(x, device=dev) for x in (q_cpu, k_cpu, v_cpu))
+    od = torch.empty_like(qd)
+    perm = any(routes)
+    if perm:
+        qp, kp, vp, op = (torch.empty_like(qd) for _ in range(4))
+
+    def e2e_step():
+        for h_, d_ in ((qh, qd), (kh, kd), (vh, vd)):
+            d_.copy_(h_, non_blocking=True)
+        if perm:
+            for a, b_ in ((qd, qp), (kd, kp), (vd, vp)):
+                S.svg_permute(a, b_, routes, g, m)
+            S.svg_attention_fwd(qp, kp, vp, op, routes, ws[0], ws[1], g, m, t, mode=mode, scratch=scratch)
+            S.svg_permute(op, od, routes, g, m, inverse=True)
+        else:
+            S.svg_attention_fwd(qd, kd, vd, od, routes, ws[0], ws[1], g, m, t, mode=mode, scratch=scratch)
+        oh.copy_(od, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    n = max(3, min(20, args.steps // 5))
+    ms = time_events(e2e_step, n, stream)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    h2d = 3 * q_cpu.numel() * 2
+    d2h = q_cpu.numel() * 2
+    return {"value": world * eff_flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

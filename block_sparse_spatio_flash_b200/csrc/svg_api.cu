@@ -1,0 +1,308 @@
+// svg_api.cu -- the extern "C" entry points of libsvgattn (declared in include/svg.h).
+//
+// Host side only: argument validation, tensor-map encoding, launch configuration. Every
+// numeric step runs in the kernels of svg_tilemap.cu, svg_permute.cu and svg_attention.cu.
+// Nothing here allocates device memory.
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "svg_common.cuh"
+
+namespace svg {
+int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* ws, cudaStream_t st);
+int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const uint8_t* h_route, svg_geom geom,
+                   svg_mask mask, int inverse, int num_sms, cudaStream_t st);
+int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st);
+}  // namespace svg
+
+using namespace svg;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Compute capability and SM count of the current device (cached per device).
+int device_info(int* num_sms) {
+  static std::mutex mu;
+  static int sms[kMaxDevices] = {0};
+  static int ok[kMaxDevices] = {0};  // 0 unknown, 1 sm_100, -1 other
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SVG_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ok[dev] == 0) {
+    int major = 0, minor = 0, n = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SVG_ERR_CUDA;
+    ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    sms[dev] = n;
+  }
+  if (ok[dev] != 1) return SVG_ERR_UNSUPPORTED;
+  if (num_sms) *num_sms = sms[dev];
+  return SVG_OK;
+}
+
+bool geom_ok(const svg_geom& g) {
+  if (g.frames < 1 || g.grid_h < 1 || g.grid_w < 1) return false;
+  const int64_t n = (int64_t)g.frames * g.grid_h * g.grid_w;
+  return n >= 1 && n <= kMaxTokens;
+}
+
+bool mask_ok(const svg_geom& g, const svg_mask& m) {
+  return m.frame_window >= 0 && m.spatial_band >= 0 && m.sink_frames >= 0 && m.sink_frames <= g.frames &&
+         (m.variant == SVG_MASK_EXACT || m.variant == SVG_MASK_ROUNDED) &&
+         (m.layout == SVG_LAYOUT_SINK_PREFIX || m.layout == SVG_LAYOUT_FULL_SPACE_MAJOR);
+}
+
+bool tile_ok(const svg_tile& t) {
+  return (t.bq == 64 || t.bq == 128 || t.bq == 256 || t.bq == 512) && (t.bk == 64 || t.bk == 128);
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [heads, tokens, d] bf16 viewed as a 3-D tensor (d, tokens, heads); box = 64 columns
+// (128 bytes, one swizzle atom wide) x box_rows rows x 1 head; rows past the end read 0.
+int encode_qkv_map(CUtensorMap* m, const void* base, int heads, int tokens, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return SVG_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)tokens, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)tokens * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SVG_OK : SVG_ERR_CUDA;
+}
+
+int check_qkvo(const void* q, const void* k, const void* v, const void* o, const float* lse, int heads,
+               int64_t tokens, int d) {
+  if (!q || !k || !v || !o) return SVG_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
+    return SVG_ERR_ARG;
+  if (heads < 1 || heads > kMaxHeads || tokens < 1 || tokens > kMaxTokens) return SVG_ERR_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  return SVG_OK;
+}
+
+int run_attention(const void* q, const void* k, const void* v, void* o, float* lse, int heads, int64_t tokens,
+                  int d, float scale, const uint8_t* h_route, const void* ws_sp, const void* ws_tm,
+                  const svg_geom* geom, const svg_mask* mask, int bq, int bk, int mode, bool dense,
+                  void* scratch, size_t scratch_bytes, int32_t* d_status, cudaStream_t st) {
+  int rc = check_qkvo(q, k, v, o, lse, heads, tokens, d);
+  if (rc) return rc;
+  if (!scratch || scratch_bytes < kScratchBytes || !aligned(scratch, 16)) return SVG_ERR_ARG;
+  if (d_status && !aligned(d_status, 4)) return SVG_ERR_ARG;
+  if (bk != 64 && bk != 128) return SVG_ERR_UNSUPPORTED;
+  int num_sms = 0;
+  rc = device_info(&num_sms);
+  if (rc) return rc;
+
+  static AttnParams P;  // large (tensor maps); built under a lock, copied by value at launch
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  memset(&P, 0, sizeof(P));
+  const int N = (int)tokens;
+  P.H = heads;
+  P.N = N;
+  P.nk = (N + bk - 1) / bk;
+  P.npairs = (N + kPairRows - 1) / kPairRows;
+  const int64_t items = (int64_t)heads * P.npairs;
+  if (items > 0x7FFFFFFF) return SVG_ERR_ARG;
+  P.n_items = (int)items;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  P.sl2 = sc * 1.4426950408889634f;
+  P.dense = dense ? 1 : 0;
+  P.naive = mode == SVG_MODE_NAIVE ? 1 : 0;
+  P.o = static_cast<__nv_bfloat16*>(o);
+  P.lse = lse;
+  P.status = d_status ? d_status : static_cast<int*>(scratch);
+  P.counter = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(scratch) + 8);
+  if (!dense) {
+    if (!h_route || !geom || !mask) return SVG_ERR_ARG;
+    if (!geom_ok(*geom) || !mask_ok(*geom, *mask)) return SVG_ERR_ARG;
+    const svg_tile t{bq, bk};
+    if (!tile_ok(t)) return SVG_ERR_UNSUPPORTED;
+    if ((int64_t)geom->frames * geom->grid_h * geom->grid_w != tokens) return SVG_ERR_ARG;
+    if (mode != SVG_MODE_SPLIT && mode != SVG_MODE_NAIVE) return SVG_ERR_ARG;
+    const TmLayout L = tm_layout(N, bq, bk);
+    const void* ws[2] = {ws_sp, ws_tm};
+    for (int h = 0; h < heads; ++h) {
+      if (h_route[h] > 1) return SVG_ERR_ARG;
+      if (h_route[h]) P.route_bits[h >> 5] |= 1u << (h & 31);
+      P.uses[h_route[h]] = 1;
+    }
+    for (int c = 0; c < 2; ++c) {
+      P.g[c] = make_geom(*geom, *mask, c);
+      if (!P.uses[c]) continue;
+      if (!ws[c] || !aligned(ws[c], 256)) return SVG_ERR_WORKSPACE;
+      const uint8_t* b = static_cast<const uint8_t*>(ws[c]);
+      P.hdr[c] = reinterpret_cast<const TmHeader*>(b);
+      P.cls[c] = b + L.cls;
+      P.pair_ptr[c] = reinterpret_cast<const uint32_t*>(b + L.pair_ptr);
+      P.pair_ent[c] = reinterpret_cast<const uint32_t*>(b + L.pair_ent);
+      P.pair_cnt[c] = reinterpret_cast<const uint32_t*>(b + L.pair_cnt);
+      P.pair_order[c] = reinterpret_cast<const uint32_t*>(b + L.pair_order);
+    }
+    P.variant = mask->variant;
+    P.bq = bq;
+    P.exp_T = geom->frames;
+    P.exp_H = geom->grid_h;
+    P.exp_W = geom->grid_w;
+    P.exp_k = mask->frame_window;
+    P.exp_b = mask->spatial_band;
+    P.exp_F0 = mask->sink_frames;
+    P.exp_variant = mask->variant;
+    P.exp_layout = mask->layout;
+    P.exp_bq = bq;
+    P.exp_bk = bk;
+  }
+  if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
+  if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, bk))) return rc;
+  if ((rc = encode_qkv_map(&P.tm_v, v, heads, N, d, bk))) return rc;
+  if (cudaMemsetAsync(scratch, 0, kScratchBytes, st) != cudaSuccess) return SVG_ERR_CUDA;
+  if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int32_t), st) != cudaSuccess) return SVG_ERR_CUDA;
+  const int grid = (int)(P.n_items < num_sms ? P.n_items : num_sms);
+  return launch_attention(P, d, bk, grid, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int svg_version(void) { return 10000; }
+
+const char* svg_error_string(int code) {
+  switch (code) {
+    case SVG_OK: return "ok";
+    case SVG_ERR_ARG: return "invalid argument (pointer, alignment, size, shape or parameter)";
+    case SVG_ERR_UNSUPPORTED: return "unsupported: needs a compute capability 10.0 (sm_100a) device, d in {64,128}, "
+                                     "bq in {64,128,256,512}, bk in {64,128}";
+    case SVG_ERR_CUDA: return "a CUDA runtime or driver call failed";
+    case SVG_ERR_TIMEOUT: return "a device pipeline wait exceeded its time limit; the kernel stopped early";
+    case SVG_ERR_WORKSPACE: return "tile-map workspace missing, too small, misaligned or built for other parameters";
+    default: return "unknown error code";
+  }
+}
+
+size_t svg_tilemap_bytes(svg_geom geom, svg_tile tile) {
+  if (!geom_ok(geom) || !tile_ok(tile)) return 0;
+  return (size_t)tm_layout((int64_t)geom.frames * geom.grid_h * geom.grid_w, tile.bq, tile.bk).total;
+}
+
+int svg_tilemap_get_layout(svg_geom geom, svg_tile tile, svg_tilemap_layout* out) {
+  if (!out || !geom_ok(geom)) return SVG_ERR_ARG;
+  if (!tile_ok(tile)) return SVG_ERR_UNSUPPORTED;
+  const TmLayout L = tm_layout((int64_t)geom.frames * geom.grid_h * geom.grid_w, tile.bq, tile.bk);
+  out->total_bytes = L.total;
+  out->cls = L.cls;
+  out->cnt = L.cnt;
+  out->row_ptr = L.row_ptr;
+  out->cols = L.cols;
+  out->pair_ptr = L.pair_ptr;
+  out->pair_ent = L.pair_ent;
+  out->pair_cnt = L.pair_cnt;
+  out->pair_order = L.pair_order;
+  out->nq = L.nq;
+  out->nk = L.nk;
+  out->npairs = L.npairs;
+  out->reserved = 0;
+  return SVG_OK;
+}
+
+int svg_build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int32_t route, void* d_ws, size_t ws_bytes,
+                      void* stream) {
+  if (!geom_ok(geom) || !mask_ok(geom, mask) || (route != SVG_ROUTE_SPATIAL && route != SVG_ROUTE_TEMPORAL))
+    return SVG_ERR_ARG;
+  if (!tile_ok(tile)) return SVG_ERR_UNSUPPORTED;
+  if (!d_ws || !aligned(d_ws, 256)) return SVG_ERR_WORKSPACE;
+  if (ws_bytes < svg_tilemap_bytes(geom, tile)) return SVG_ERR_WORKSPACE;
+  int rc = device_info(nullptr);
+  if (rc) return rc;
+  return build_tilemap(geom, mask, tile, route, d_ws, static_cast<cudaStream_t>(stream));
+}
+
+int svg_tilemap_summary(const void* d_ws, svg_tilemap_summary_t* h_out, void* stream) {
+  if (!d_ws || !h_out || !aligned(d_ws, 256)) return SVG_ERR_ARG;
+  TmHeader h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, d_ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SVG_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SVG_ERR_CUDA;
+  if (h.magic != kTmMagic) return SVG_ERR_WORKSPACE;
+  h_out->retained_exact = h.retained_exact;
+  h_out->retained_map = h.retained_map;
+  h_out->n_full = h.n_full;
+  h_out->n_boundary = h.n_boundary;
+  h_out->n_empty = h.n_empty;
+  h_out->visited_area = h.visited_area;
+  h_out->pair_entries = h.pair_entries;
+  h_out->pair_half_tiles = h.pair_half_tiles;
+  return SVG_OK;
+}
+
+int svg_permute(const void* d_in, void* d_out, int32_t heads, int64_t tokens, int32_t d, const uint8_t* h_route,
+                svg_geom geom, svg_mask mask, int32_t inverse, void* stream) {
+  if (!d_in || !d_out || !h_route || !aligned(d_in, 16) || !aligned(d_out, 16)) return SVG_ERR_ARG;
+  if (heads < 1 || heads > kMaxHeads || !geom_ok(geom) || !mask_ok(geom, mask)) return SVG_ERR_ARG;
+  if ((int64_t)geom.frames * geom.grid_h * geom.grid_w != tokens) return SVG_ERR_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  if (inverse != 0 && inverse != 1) return SVG_ERR_ARG;
+  const uint8_t* a = static_cast<const uint8_t*>(d_in);
+  const uint8_t* b = static_cast<const uint8_t*>(d_out);
+  const size_t bytes = (size_t)heads * tokens * d * 2;
+  if (a < b + bytes && b < a + bytes) return SVG_ERR_ARG;  // must not overlap
+  for (int h = 0; h < heads; ++h)
+    if (h_route[h] > 1) return SVG_ERR_ARG;
+  int num_sms = 0;
+  int rc = device_info(&num_sms);
+  if (rc) return rc;
+  return launch_permute(d_in, d_out, heads, tokens, d, h_route, geom, mask, inverse, num_sms,
+                        static_cast<cudaStream_t>(stream));
+}
+
+size_t svg_attention_scratch_bytes(void) { return kScratchBytes; }
+
+int svg_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,
+                      int64_t tokens, int32_t d, float scale, const uint8_t* h_route, const void* d_ws_spatial,
+                      const void* d_ws_temporal, svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
+                      void* d_scratch, size_t scratch_bytes, int32_t* d_status, void* stream) {
+  return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
+                       tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int svg_dense_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,
+                            int64_t tokens, int32_t d, float scale, int32_t bk, void* d_scratch, size_t scratch_bytes,
+                            int32_t* d_status, void* stream) {
+  return run_attention(q, k, v, o, lse, heads, tokens, d, scale, nullptr, nullptr, nullptr, nullptr, nullptr, 0, bk,
+                       SVG_MODE_SPLIT, true, d_scratch, scratch_bytes, d_status, static_cast<cudaStream_t>(stream));
+}
+
+int svg_read_status(const void* d_scratch_or_status, int32_t* h_status, void* stream) {
+  if (!d_scratch_or_status || !h_status || !aligned(d_scratch_or_status, 4)) return SVG_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(h_status, d_scratch_or_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SVG_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
+}
+
+}  // extern "C"

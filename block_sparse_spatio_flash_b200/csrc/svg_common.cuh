@@ -1,0 +1,360 @@
+// svg_common.cuh -- shared definitions of the libsvgattn CUDA sources (sm_100a only).
+//
+//  * MaskGeom: the spatial / temporal masks of the Sparse-VideoGen routing as described in
+//    "Accelerating Spatio-Temporal Attention for Video Diffusion on TPUs" ("Sparse Attention
+//    Patterns": spatial heads look at the same or nearby frames, temporal heads at a narrow
+//    spatial region across frames; "Interesting facts": both keep the first frame as a sink,
+//    temporal heads need their own token order), expressed in POSITION space: for a query at
+//    position p the kept keys are [0, sink_end) U [lo(p), hi(p)) U (periodic sink), a form that
+//    makes tile classification O(1) per row and boundary masking a few compares per element.
+//  * TmHeader: the record at the start of a tile-map workspace.
+//  * Thin inline-PTX wrappers for mbarrier, TMA (cp.async.bulk.tensor) and tcgen05.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/svg.h"
+
+namespace svg {
+
+constexpr uint32_t kTmMagic = 0x53564731u;  // "SVG1"
+constexpr int kMaxHeads = 4096;
+constexpr int64_t kMaxTokens = 1 << 22;
+constexpr int kPairRows = 256;  // query rows per execution item: two 128-row halves
+constexpr int kHalfRows = 128;
+
+// ---------------------------------------------------------------------------------------
+// Mask geometry in position space.
+struct MaskGeom {
+  int T, S, N;        // frames, tokens per frame, tokens
+  int k, b, F0;       // frame window, spatial band, sink frames
+  int route, layout;  // SVG_ROUTE_*, SVG_LAYOUT_* (layout only matters for temporal heads)
+};
+
+__host__ __device__ inline MaskGeom make_geom(const svg_geom& g, const svg_mask& m, int route) {
+  MaskGeom r;
+  r.T = g.frames;
+  r.S = g.grid_h * g.grid_w;
+  r.N = r.T * r.S;
+  r.k = m.frame_window;
+  r.b = m.spatial_band;
+  r.F0 = m.sink_frames;
+  r.route = route;
+  r.layout = m.layout;
+  return r;
+}
+
+// True when the head's sink is the periodic set {c : c mod T < F0} (fully space-major order).
+__host__ __device__ inline bool periodic_sink(const MaskGeom& g) {
+  return g.route == SVG_ROUTE_TEMPORAL && g.layout == SVG_LAYOUT_FULL_SPACE_MAJOR && g.F0 > 0;
+}
+
+// End of the contiguous sink prefix [0, sink_end) of key positions.
+__host__ __device__ inline int sink_end(const MaskGeom& g) {
+  if (g.route == SVG_ROUTE_TEMPORAL && g.layout == SVG_LAYOUT_FULL_SPACE_MAJOR) return 0;
+  return g.F0 * g.S;
+}
+
+// (frame, patch) of the token at position p of this head's order.
+__host__ __device__ inline void pos_to_ts(const MaskGeom& g, int p, int& t, int& s) {
+  if (g.route == SVG_ROUTE_SPATIAL) {
+    t = p / g.S;
+    s = p - t * g.S;
+    return;
+  }
+  if (g.layout == SVG_LAYOUT_FULL_SPACE_MAJOR) {
+    s = p / g.T;
+    t = p - s * g.T;
+    return;
+  }
+  const int pre = g.F0 * g.S;
+  if (p < pre) {
+    t = p / g.S;
+    s = p - t * g.S;
+    return;
+  }
+  const int q = p - pre, tr = g.T - g.F0;
+  s = q / tr;
+  t = g.F0 + (q - s * tr);
+}
+
+// Position of token (t, s) in this head's order.
+__host__ __device__ inline int ts_to_pos(const MaskGeom& g, int t, int s) {
+  if (g.route == SVG_ROUTE_SPATIAL) return t * g.S + s;
+  if (g.layout == SVG_LAYOUT_FULL_SPACE_MAJOR) return s * g.T + t;
+  if (t < g.F0) return t * g.S + s;
+  return g.F0 * g.S + s * (g.T - g.F0) + (t - g.F0);
+}
+
+// Window / band part of the kept key positions of the query at position p: [lo, hi).
+// Spatial: frames [t-k, t+k] are contiguous in frame-major order. Temporal: patches
+// [s-b, s+b] are contiguous in the space-major part of the order (and the sink-frame copies
+// of those patches are inside the sink anyway).
+__host__ __device__ inline void row_interval(const MaskGeom& g, int p, int& lo, int& hi) {
+  int t, s;
+  pos_to_ts(g, p, t, s);
+  if (g.route == SVG_ROUTE_SPATIAL) {
+    const int f0 = t - g.k < 0 ? 0 : t - g.k;
+    const int f1 = t + g.k > g.T - 1 ? g.T - 1 : t + g.k;
+    lo = f0 * g.S;
+    hi = (f1 + 1) * g.S;
+    return;
+  }
+  const int s0 = s - g.b < 0 ? 0 : s - g.b;
+  const int s1 = s + g.b > g.S - 1 ? g.S - 1 : s + g.b;
+  if (g.layout == SVG_LAYOUT_FULL_SPACE_MAJOR) {
+    lo = s0 * g.T;
+    hi = (s1 + 1) * g.T;
+  } else {
+    const int pre = g.F0 * g.S, tr = g.T - g.F0;
+    lo = pre + s0 * tr;
+    hi = pre + (s1 + 1) * tr;
+  }
+}
+
+__host__ __device__ inline int ilen(int a0, int a1) { return a1 > a0 ? a1 - a0 : 0; }
+
+// #{c in [0, x) : c mod T < F0}
+__host__ __device__ inline int periodic_prefix(const MaskGeom& g, int x) {
+  const int q = x / g.T, r = x - q * g.T;
+  return q * g.F0 + (r < g.F0 ? r : g.F0);
+}
+
+// Kept keys of a query row (interval [lo, hi)) inside key positions [c0, c1).
+__host__ __device__ inline int row_kept_in(const MaskGeom& g, int lo, int hi, int c0, int c1) {
+  const int b0 = lo > c0 ? lo : c0, b1 = hi < c1 ? hi : c1;
+  int n = ilen(b0, b1);
+  const int se = sink_end(g);
+  if (se > 0) n += ilen(c0, se < c1 ? se : c1) - ilen(b0, se < b1 ? se : b1);
+  if (periodic_sink(g)) {
+    n += periodic_prefix(g, c1) - periodic_prefix(g, c0);
+    if (b1 > b0) n -= periodic_prefix(g, b1) - periodic_prefix(g, b0);
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------------------------------
+// Tile-map workspace record (offset 0 of the workspace, 256 bytes).
+struct TmHeader {
+  uint32_t magic, version;
+  int32_t T, H, W, route, k, b, F0, variant, layout, bq, bk, nq, nk, npairs, N, pad0;
+  unsigned long long retained_exact, retained_map, n_full, n_boundary, n_empty, visited_area,
+      pair_entries, pair_half_tiles;
+};
+static_assert(sizeof(TmHeader) <= 256, "header must fit in 256 bytes");
+
+struct TmLayout {
+  uint64_t total, cls, cnt, row_ptr, cols, pair_ptr, pair_ent, pair_cnt, pair_order;
+  int nq, nk, npairs;
+};
+
+inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+inline TmLayout tm_layout(int64_t N, int bq, int bk) {
+  TmLayout L;
+  L.nq = (int)((N + bq - 1) / bq);
+  L.nk = (int)((N + bk - 1) / bk);
+  L.npairs = (int)((N + kPairRows - 1) / kPairRows);
+  const uint64_t tiles = (uint64_t)L.nq * L.nk;
+  uint64_t off = 256;
+  L.cls = off;        off = align_up(off + tiles, 256);
+  L.cnt = off;        off = align_up(off + 4 * tiles, 256);
+  L.row_ptr = off;    off = align_up(off + 4 * (uint64_t)(L.nq + 1), 256);
+  L.cols = off;       off = align_up(off + 4 * tiles, 256);
+  L.pair_ptr = off;   off = align_up(off + 4 * (uint64_t)(L.npairs + 1), 256);
+  L.pair_ent = off;   off = align_up(off + 4 * (uint64_t)L.npairs * L.nk, 256);
+  L.pair_cnt = off;   off = align_up(off + 8 * (uint64_t)L.npairs, 256);
+  L.pair_order = off; off = align_up(off + 4 * (uint64_t)L.npairs, 256);
+  L.total = off;
+  return L;
+}
+
+// Execution-list entry: kt | flagA << 28 | flagB << 30.
+enum : uint32_t { kFlagSkip = 0, kFlagFull = 1, kFlagMasked = 2, kFlagBounds = 3 };
+__host__ __device__ inline uint32_t ent_kt(uint32_t e) { return e & 0x0FFFFFFFu; }
+__host__ __device__ inline uint32_t ent_flag(uint32_t e, int half) { return (e >> (28 + 2 * half)) & 3u; }
+
+// Scratch of the attention entry points: [0] status, [1] reserved, [2] work counter.
+constexpr size_t kScratchBytes = 256;
+
+// Launch parameters of the attention kernel (filled on the host, read on the device).
+struct AttnParams {
+  CUtensorMap tm_q, tm_k, tm_v;
+  __nv_bfloat16* o;
+  float* lse;
+  int H, N, npairs, nk, n_items;
+  float sl2;  // scale * log2(e)
+  int dense, naive, variant, bq;
+  MaskGeom g[2];
+  const TmHeader* hdr[2];
+  const uint8_t* cls[2];
+  const uint32_t* pair_ptr[2];
+  const uint32_t* pair_ent[2];
+  const uint32_t* pair_cnt[2];
+  const uint32_t* pair_order[2];
+  int uses[2];
+  int exp_T, exp_H, exp_W, exp_k, exp_b, exp_F0, exp_variant, exp_layout, exp_bq, exp_bk;
+  int* status;
+  unsigned int* counter;
+  uint32_t route_bits[kMaxHeads / 32];
+};
+
+// ---------------------------------------------------------------------------------------
+// PTX wrappers.
+#if defined(__CUDACC__)
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// 3-D tiled TMA load global -> shared, completion counted on `bar` (bytes). No multicast.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// tcgen05 (5th-generation tensor cores, TMEM accumulators), CTA group 1.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// mbarrier arrives once every tcgen05 op issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+#define SVG_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
+                  "=r"(r[i + 6]), "=r"(r[i + 7])
+#define SVG_W8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
+                  "r"(r[i + 6]), "r"(r[i + 7])
+#define SVG_D8(i) "+r"(r[i + 0]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), \
+                  "+r"(r[i + 6]), "+r"(r[i + 7])
+
+// 32 lanes x 32 columns of 32 bits: thread i of the warp receives lane (base_lane + i),
+// columns [col, col+32). Results are valid only after tmem_ld_fence32 on the same array.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : SVG_R8(0), SVG_R8(8), SVG_R8(16), SVG_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+// Orders later uses of r[0..32) after the completion wait (a data dependency through asm).
+__device__ __forceinline__ void tmem_ld_fence32(uint32_t* r) {
+  asm volatile("" : SVG_D8(0), SVG_D8(8), SVG_D8(16), SVG_D8(24) : : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      SVG_W8(0), SVG_W8(8), SVG_W8(16), SVG_W8(24)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      SVG_W8(0), SVG_W8(8)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 format): start>>4 [0,14), LBO>>4 [16,30),
+// SBO>>4 [32,46), version 1 at bit 46, layout type [61,64) (2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n, bool b_mn_major) {
+  return (1u << 4)                      // D format fp32
+         | (1u << 7)                    // A format bf16
+         | (1u << 10)                   // B format bf16
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(n >> 3) << 17)   // N / 8
+         | ((uint32_t)(128 >> 4) << 24);  // M / 16
+}
+#endif  // __CUDACC__
+
+}  // namespace svg

@@ -1,0 +1,189 @@
+/*
+ * svg.h -- C ABI of libsvgattn: block-sparse spatio-temporal attention forward on B200.
+ *
+ * The operation ("Accelerating Spatio-Temporal Attention for Video Diffusion on TPUs",
+ * Google Developers Blog case study, as summarised on the three pages on the subject):
+ * video-diffusion attention heads are routed either to a SPATIAL mask (keys in the same or
+ * nearby frames) or to a TEMPORAL mask (keys in a narrow spatial region across all frames),
+ * both keeping full attention to the first frame as a sink ("Sparse Attention Patterns";
+ * "Interesting facts"). The kernel tiles the query x key plane, skips empty tiles, runs full
+ * tiles without evaluating the mask and masks only boundary tiles ("Efficient Kernel
+ * Implementation", tile-aware masking). Temporal heads are reordered space-major first so
+ * their mask becomes regular ("Interesting facts": token ordering). An optional tile-aligned
+ * variant rounds the mask to whole tiles (summary; "What changed").
+ *
+ * Mask, on ORIGINAL token identities (token i = t*S + s, frame t, flattened patch
+ * s = y*grid_w + x, S = grid_h*grid_w, N = frames*S):
+ *   spatial:  keep(i,j) <=> |t(i)-t(j)| <= frame_window  or  t(j) < sink_frames
+ *   temporal: keep(i,j) <=> |s(i)-s(j)| <= spatial_band  or  t(j) < sink_frames
+ * Token order (position of token (t,s)) used by a head's Q/K/V/O rows on the device:
+ *   spatial heads:  t*S + s                                   (frame-major, unchanged)
+ *   temporal heads, SVG_LAYOUT_SINK_PREFIX (F0 = sink_frames):
+ *                   t <  F0: t*S + s ;  t >= F0: F0*S + s*(frames-F0) + (t-F0)
+ *   temporal heads, SVG_LAYOUT_FULL_SPACE_MAJOR: s*frames + t
+ * Tiles are bq x bk blocks of the (query position, key position) plane; a tile is FULL if
+ * every in-range pair is kept, EMPTY if none is, BOUNDARY otherwise. The rounded variant
+ * keeps a whole tile iff 2*kept >= in-range area, and drops it otherwise.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are contiguous [heads, tokens, d] bf16 (raw 16-bit patterns), device memory,
+ *     16-byte aligned. The caller owns and allocates every buffer; the library allocates no
+ *     device memory on any call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). All device
+ *     work is enqueued asynchronously on it; only svg_tilemap_summary and svg_read_status
+ *     synchronise (that stream only).
+ *   - Host arrays (`h_route`) are read during the call and may be freed when it returns.
+ *   - Return value: SVG_OK (0) or a negative SVG_ERR_* code; nothing is enqueued when an
+ *     argument check fails. Errors detected on the device (a wait that timed out, a tile map
+ *     built for other parameters) are written to the status word (see svg_read_status).
+ *   - Requires a compute capability 10.0 device (B200, sm_100a); otherwise
+ *     SVG_ERR_UNSUPPORTED.
+ */
+#ifndef SVG_H_
+#define SVG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SVG_OK 0
+#define SVG_ERR_ARG (-1)          /* bad pointer, size, shape or parameter combination */
+#define SVG_ERR_UNSUPPORTED (-2)  /* not an sm_100 device, or d / tile shape not supported */
+#define SVG_ERR_CUDA (-3)         /* a CUDA runtime/driver call failed */
+#define SVG_ERR_TIMEOUT (-4)      /* device status: a pipeline wait exceeded its time limit */
+#define SVG_ERR_WORKSPACE (-5)    /* workspace too small, or built for other parameters */
+
+enum { SVG_ROUTE_SPATIAL = 0, SVG_ROUTE_TEMPORAL = 1 };
+enum { SVG_MASK_EXACT = 0, SVG_MASK_ROUNDED = 1 };
+enum { SVG_LAYOUT_SINK_PREFIX = 0, SVG_LAYOUT_FULL_SPACE_MAJOR = 1 };
+/* SPLIT: full tiles unmasked, boundary tiles element-masked (the pages' fast path).
+ * NAIVE: every visited tile element-masked (the pages' slower first sparse kernel). */
+enum { SVG_MODE_SPLIT = 0, SVG_MODE_NAIVE = 1 };
+
+typedef struct { int32_t frames, grid_h, grid_w; } svg_geom;
+
+typedef struct {
+    int32_t frame_window;  /* k >= 0: spatial heads keep key frames with |t_q - t_k| <= k   */
+    int32_t spatial_band;  /* b >= 0: temporal heads keep keys with |s_q - s_k| <= b        */
+    int32_t sink_frames;   /* F0 in [0, frames]: keys of frames [0, F0) are always kept      */
+    int32_t variant;       /* SVG_MASK_EXACT or SVG_MASK_ROUNDED                            */
+    int32_t layout;        /* token order of temporal heads (SVG_LAYOUT_*)                  */
+} svg_mask;
+
+typedef struct { int32_t bq, bk; } svg_tile;   /* bq in {64,128,256,512}, bk in {64,128} */
+
+/* Byte offsets of the arrays inside a tile-map workspace (see svg_build_tilemap). */
+typedef struct {
+    uint64_t total_bytes;
+    uint64_t cls;         /* uint8  [nq*nk]   class per tile: 0 empty, 1 full, 2 boundary   */
+    uint64_t cnt;         /* uint32 [nq*nk]   EXACT retained pairs per tile                 */
+    uint64_t row_ptr;     /* uint32 [nq+1]    CSR offsets of visited tiles per q-tile        */
+    uint64_t cols;        /* uint32 [...]     kt | class << 30, ascending kt                 */
+    uint64_t pair_ptr;    /* uint32 [np+1]    offsets of the 256-row execution lists         */
+    uint64_t pair_ent;    /* uint32 [...]     kt | flagA << 28 | flagB << 30                  */
+    uint64_t pair_cnt;    /* uint32 [2*np]    active entries of half 0 / half 1 of each pair  */
+    uint64_t pair_order;  /* uint32 [np]      pairs by descending work, ties by index         */
+    int32_t nq, nk, npairs, reserved;
+} svg_tilemap_layout;
+
+/* Totals of one built tile map (svg_tilemap_summary). */
+typedef struct {
+    uint64_t retained_exact;  /* kept pairs of the exact mask (layout-independent)        */
+    uint64_t retained_map;    /* kept pairs of the map's own mask (= exact, or rounded)    */
+    uint64_t n_full, n_boundary, n_empty;   /* tile classes of the map                      */
+    uint64_t visited_area;    /* in-range pairs inside non-empty tiles                     */
+    uint64_t pair_entries;    /* entries of all 256-row execution lists                    */
+    uint64_t pair_half_tiles; /* active (entry, half) combinations: MMA work units          */
+} svg_tilemap_summary_t;
+
+/*
+ * Size of the tile-map workspace for ONE route class (all heads of a class share it):
+ * the largest the map can need for this geometry and tile shape. Returns 0 on bad args.
+ */
+size_t svg_tilemap_bytes(svg_geom geom, svg_tile tile);
+
+/* Fills *out with the byte offsets used by svg_build_tilemap. Host-only, no device work. */
+int svg_tilemap_get_layout(svg_geom geom, svg_tile tile, svg_tilemap_layout *out);
+
+/*
+ * Classifies every (query tile, key tile) pair of one route class as full / boundary /
+ * empty (rounded variant: full / empty), counts retained pairs per tile exactly, and
+ * builds: the per-q-tile CSR list of visited tiles; the execution lists used by
+ * svg_attention_fwd (one per 256-query-row pair of 128-row halves, with per-half flags
+ * 0 skip, 1 full, 2 masked, 3 full but key range past the sequence end); and the pair
+ * order by descending work used by its persistent scheduler. Integer work only.
+ *   d_ws: device buffer of at least svg_tilemap_bytes(geom, tile) bytes, 256-B aligned;
+ *         written entirely by this call (also records the parameters it was built for).
+ * Errors: SVG_ERR_ARG (bad geometry/mask/route), SVG_ERR_UNSUPPORTED (tile shape),
+ *         SVG_ERR_WORKSPACE (ws_bytes too small), SVG_ERR_CUDA (launch failure).
+ */
+int svg_build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int32_t route,
+                      void *d_ws, size_t ws_bytes, void *stream);
+
+/* Copies the totals of a built map to *h_out. Synchronises `stream`. */
+int svg_tilemap_summary(const void *d_ws, svg_tilemap_summary_t *h_out, void *stream);
+
+/*
+ * Token permutation of a [heads, tokens, d] bf16 tensor (d_in != d_out, no overlap).
+ * inverse = 0: out[h][pi_h(i)] = in[h][i]   (original order -> the head's order)
+ * inverse = 1: out[h][i] = in[h][pi_h(i)]   (the head's order -> original order)
+ * pi_h is the identity for spatial heads (rows are still copied) and the temporal order
+ * selected by mask.layout / mask.sink_frames for temporal heads. h_route: host uint8
+ * [heads], SVG_ROUTE_*. tokens must equal frames*grid_h*grid_w; d in {64, 128};
+ * heads <= 4096. Pure data movement (HBM-bound).
+ */
+int svg_permute(const void *d_in, void *d_out, int32_t heads, int64_t tokens, int32_t d,
+                const uint8_t *h_route, svg_geom geom, svg_mask mask, int32_t inverse,
+                void *stream);
+
+/* Bytes of scratch svg_attention_fwd / svg_dense_attention_fwd need (scheduler counter
+ * and status word). The calls clear it themselves. */
+size_t svg_attention_scratch_bytes(void);
+
+/*
+ * Block-sparse attention forward, flash-style (online softmax), tensor cores (tcgen05).
+ *   q, k, v: [heads, tokens, d] bf16, each head's rows in that head's token order
+ *            (svg_permute, inverse = 0, for temporal heads).
+ *   o:       [heads, tokens, d] bf16 output in the same order (svg_permute inverse = 1
+ *            restores original order for temporal heads).
+ *   lse:     nullable fp32 [heads, tokens]: natural-log sum of exp of the kept scaled
+ *            scores per row (-inf and O = 0 for a row with no kept key).
+ *   scale:   softmax scale; <= 0 selects 1/sqrt(d).
+ *   h_route: host uint8 [heads] route per head; heads <= 4096.
+ *   d_ws_spatial / d_ws_temporal: tile maps built by svg_build_tilemap for the route class
+ *            with the same geom, mask and tile (may be NULL if no head uses that class).
+ *   mode:    SVG_MODE_SPLIT or SVG_MODE_NAIVE.
+ *   d_scratch: device buffer of svg_attention_scratch_bytes() bytes (cleared by the call).
+ *   d_status:  nullable device int32; receives 0 or a negative SVG_ERR_* code detected on
+ *              the device. When NULL, the status word inside d_scratch is used.
+ * d in {64, 128}; tile.bk selects the key-tile width the kernel streams.
+ */
+int svg_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                      int32_t heads, int64_t tokens, int32_t d, float scale,
+                      const uint8_t *h_route, const void *d_ws_spatial, const void *d_ws_temporal,
+                      svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
+                      void *d_scratch, size_t scratch_bytes, int32_t *d_status, void *stream);
+
+/* Dense attention forward (every pair kept) with the same kernel and scheduler; the
+ * in-repo baseline. Arguments as in svg_attention_fwd; bk in {64, 128}. */
+int svg_dense_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int32_t heads, int64_t tokens, int32_t d, float scale, int32_t bk,
+                            void *d_scratch, size_t scratch_bytes, int32_t *d_status,
+                            void *stream);
+
+/* Reads the device status word of a scratch buffer (or d_status). Synchronises `stream`. */
+int svg_read_status(const void *d_scratch_or_status, int32_t *h_status, void *stream);
+
+/* Static description of an error code. */
+const char *svg_error_string(int code);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int svg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVG_H_ */

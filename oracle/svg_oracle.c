@@ -171,6 +171,13 @@ void or_attention_rows(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
                        const int64_t *rows, int64_t n_rows, double *out, double *lse) {
     int64_t nk = (N + bk - 1) / bk;
     int64_t *pi = NULL;
+    /* widen K and V once (exact), so the row loops below read doubles */
+    double *kd = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    double *vd = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    for (int64_t x = 0; x < N * d; ++x) {
+        kd[x] = bf16_to_f64(kk[x]);
+        vd[x] = bf16_to_f64(v[x]);
+    }
     if (mask_kind == 1) {
         pi = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
         or_perm_table(route, layout, T, S, F0, pi);
@@ -194,7 +201,7 @@ void or_attention_rows(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
                 kp[j] = (unsigned char)keep;
                 if (!keep) continue;
                 double dot = 0.0;
-                for (int64_t x = 0; x < d; ++x) dot += qrow[x] * bf16_to_f64(kk[j * d + x]);
+                for (int64_t x = 0; x < d; ++x) dot += qrow[x] * kd[j * d + x];
                 sc[j] = scale * dot;
                 if (sc[j] > m) m = sc[j];
             }
@@ -205,7 +212,7 @@ void or_attention_rows(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
                     if (!kp[j]) continue;
                     double p = exp(sc[j] - m);
                     l += p;
-                    for (int64_t x = 0; x < d; ++x) acc[x] += p * bf16_to_f64(v[j * d + x]);
+                    for (int64_t x = 0; x < d; ++x) acc[x] += p * vd[j * d + x];
                 }
             }
             for (int64_t x = 0; x < d; ++x) out[r * d + x] = l > 0.0 ? acc[x] / l : 0.0;
@@ -213,7 +220,7 @@ void or_attention_rows(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
         }
         free(qrow); free(sc); free(kp); free(acc);
     }
-    free(pi);
+    free(pi); free(kd); free(vd);
 }
 
 /* Threads the OpenMP runtime will use (reported next to oracle timings). */

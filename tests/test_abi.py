@@ -1,0 +1,120 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point that
+include/svg.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "svg.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(svg_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def svg():
+    from block_sparse_spatio_flash_b200 import build
+    build.build()
+    from block_sparse_spatio_flash_b200 import svg as mod
+    return mod
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("svg_build_tilemap", "svg_permute", "svg_attention_fwd", "svg_dense_attention_fwd",
+              "svg_tilemap_bytes", "svg_error_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(svg):
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_library_has_no_torch_dependency(svg):
+    import subprocess
+    out = subprocess.run(["ldd", svg.LIB_PATH], capture_output=True, text=True).stdout
+    assert "torch" not in out and "c10" not in out
+
+
+def test_error_strings(svg):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert svg.svg_error_string(code)
+    assert "unknown" in svg.svg_error_string(-99)
+    assert svg.svg_version() >= 10000
+
+
+def test_tilemap_layout_sizes(svg):
+    g = svg.make_geom(21, 45, 80)
+    for bq, bk in [(128, 128), (256, 64), (512, 128), (64, 64)]:
+        t = svg.make_tile(bq, bk)
+        L = svg.svg_tilemap_get_layout(g, t)
+        n = 21 * 45 * 80
+        assert L.nq == -(-n // bq) and L.nk == -(-n // bk) and L.npairs == -(-n // 256)
+        assert L.total_bytes == svg.svg_tilemap_bytes(g, t)
+        offs = [L.cls, L.cnt, L.row_ptr, L.cols, L.pair_ptr, L.pair_ent, L.pair_cnt, L.pair_order]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert L.cnt - L.cls >= L.nq * L.nk and L.pair_ent - L.pair_ptr >= 4 * (L.npairs + 1)
+        assert L.total_bytes >= L.pair_order + 4 * L.npairs
+
+
+def test_bad_tile_and_geometry_rejected(svg):
+    g = svg.make_geom(4, 8, 16)
+    assert svg.svg_tilemap_bytes(g, svg.make_tile(96, 64)) == 0
+    assert svg.svg_tilemap_bytes(svg.make_geom(0, 8, 16), svg.make_tile(64, 64)) == 0
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    m = svg.make_mask(1, 16)
+    # bad route / mask / tile / workspace: rejected before any device work
+    assert lib.svg_build_tilemap(g, m, svg.make_tile(64, 64), 2, ctypes.c_void_p(256), 1 << 30, None) == -1
+    assert lib.svg_build_tilemap(g, svg.make_mask(-1, 16), svg.make_tile(64, 64), 0,
+                                 ctypes.c_void_p(256), 1 << 30, None) == -1
+    assert lib.svg_build_tilemap(g, svg.make_mask(1, 16, sink_frames=5), svg.make_tile(64, 64), 0,
+                                 ctypes.c_void_p(256), 1 << 30, None) == -1
+    assert lib.svg_build_tilemap(g, m, svg.make_tile(64, 32), 0, ctypes.c_void_p(256), 1 << 30, None) == -2
+    assert lib.svg_build_tilemap(g, m, svg.make_tile(64, 64), 0, None, 1 << 30, None) == -5
+    assert lib.svg_build_tilemap(g, m, svg.make_tile(64, 64), 0, ctypes.c_void_p(256), 16, None) == -5
+    assert lib.svg_build_tilemap(g, m, svg.make_tile(64, 64), 0, ctypes.c_void_p(257), 1 << 30, None) == -5
+
+
+def test_attention_argument_checks(svg):
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    g, m, t = svg.make_geom(4, 8, 16), svg.make_mask(1, 16), svg.make_tile(64, 64)
+    routes = (ctypes.c_uint8 * 2)(0, 1)
+    p = ctypes.c_void_p(1 << 20)
+    f = lib.svg_attention_fwd
+    f.argtypes = svg._sig["svg_attention_fwd"][1]
+    # null tensors, misaligned tensors, bad head count, bad d
+    assert f(None, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -1
+    assert f(ctypes.c_void_p((1 << 20) + 2), p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256,
+             None, None) == -1
+    assert f(p, p, p, p, None, 0, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -1
+    assert f(p, p, p, p, None, 2, 512, 96, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -2
+    # scratch missing or too small
+    assert f(p, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, None, 256, None, None) == -1
+    assert f(p, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 8, None, None) == -1
+    d = lib.svg_dense_attention_fwd
+    d.argtypes = svg._sig["svg_dense_attention_fwd"][1]
+    assert d(p, p, p, None, None, 2, 512, 64, 0.0, 128, p, 256, None, None) == -1
+    assert d(p, p, p, p, None, 2, 512, 64, 0.0, 32, p, 256, None, None) == -2
+
+
+def test_permute_argument_checks(svg):
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    f = lib.svg_permute
+    f.argtypes = svg._sig["svg_permute"][1]
+    g, m = svg.make_geom(4, 8, 16), svg.make_mask(1, 16)
+    routes = (ctypes.c_uint8 * 2)(0, 1)
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 30)
+    assert f(a, b, 2, 511, 64, routes, g, m, 0, None) == -1           # tokens != frames*h*w
+    assert f(a, a, 2, 512, 64, routes, g, m, 0, None) == -1           # in == out
+    assert f(a, b, 2, 512, 48, routes, g, m, 0, None) == -2           # d
+    assert f(a, b, 2, 512, 64, routes, g, m, 2, None) == -1           # inverse flag
+    bad = (ctypes.c_uint8 * 2)(0, 7)
+    assert f(a, b, 2, 512, 64, bad, g, m, 0, None) == -1              # route value

@@ -1,0 +1,286 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tile maps, retained counts and permutations are compared bit for bit; attention outputs
+within relative L2 <= 1e-2 and max-abs <= 2e-2 per head (LSE within 5e-3), on every row for
+small problems and on seeded sampled rows (plus the ragged tail) for the pages' sizes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_spatio_flash_b200 import synthetic as syn
+from tests import gpu_path as gp
+from tests.test_oracle_pins import closed_form_spatial, closed_form_temporal
+
+pytestmark = pytest.mark.gpu
+
+MEDIUM = syn.Workload("medium_1200", frames=5, grid_h=12, grid_w=20, routes=(0, 1, 0, 1), d=128,
+                      frame_window=1, spatial_band=20, bq=128, bk=128)
+
+
+@pytest.fixture(scope="module")
+def S():
+    from block_sparse_spatio_flash_b200 import build
+    build.build()
+    return gp.svg()
+
+
+def u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def expected_pair_entries(cls, N, bq, bk):
+    """Execution lists derived from the class map (flags: 0 skip, 1 full, 2 masked, 3 full but
+    ragged key tile). A 128-row half combines the classes of the q-tiles it overlaps."""
+    nq, nk = cls.shape
+    npairs = -(-N // 256)
+    ragged = np.zeros(nk, dtype=bool)
+    if N % bk:
+        ragged[-1] = True
+    ents, cnts = [], []
+    for p in range(npairs):
+        flags = []
+        for h in range(2):
+            r0 = 256 * p + 128 * h
+            if r0 >= N:
+                flags.append(np.zeros(nk, dtype=np.uint32))
+                continue
+            r1 = min(N, r0 + 128)
+            cs = cls[r0 // bq: (r1 - 1) // bq + 1]
+            anyk = (cs != 0).any(axis=0)
+            allf = (cs == 1).all(axis=0)
+            f = np.where(~anyk, 0, np.where(allf, np.where(ragged, 3, 1), 2)).astype(np.uint32)
+            flags.append(f)
+        act = (flags[0] | flags[1]) != 0
+        kts = np.nonzero(act)[0].astype(np.uint32)
+        ents.append(kts | (flags[0][act] << 28) | (flags[1][act] << 30))
+        cnts.append((int((flags[0] != 0).sum()), int((flags[1] != 0).sum())))
+    return ents, cnts
+
+
+def check_tilemap(S, w, route, variant, bq, bk, qts=None):
+    g, m, t = gp.geom_mask_tile(w, variant, bq, bk)
+    ws = S.alloc_workspace(g, t)
+    S.svg_build_tilemap(g, m, t, route, ws)
+    summ = S.svg_tilemap_summary(ws)
+    A = S.tilemap_arrays(ws, g, t)
+    N = w.tokens
+    cls = A["cls"].cpu().numpy()
+    cnt = u32(A["cnt"]).reshape(A["nq"], A["nk"])
+    full = qts is None
+    qts = np.arange(A["nq"]) if qts is None else np.asarray(qts)
+    ocnt, ocls = oracle.tile_counts(route, w.layout, w.frames, w.frame_size, w.frame_window, w.spatial_band,
+                                    w.sink_frames, bq, bk, qts=qts)
+    area = oracle.tile_areas(N, bq, bk)
+    if variant == syn.MASK_ROUNDED:
+        ocls = oracle.rounded_classes(ocnt, area[qts])
+    assert np.array_equal(cnt[qts], ocnt)
+    assert np.array_equal(cls[qts], ocls)
+    # totals: exact count of the whole map equals the closed form of the mask
+    if route == 0:
+        closed = closed_form_spatial(w.frames, w.frame_size, w.frame_window, w.sink_frames)
+    else:
+        closed = closed_form_temporal(w.frames, w.frame_size, w.spatial_band, w.sink_frames)
+    assert summ.retained_exact == closed == int(cnt.astype(np.int64).sum())
+    assert summ.n_full == int((cls == 1).sum()) and summ.n_boundary == int((cls == 2).sum())
+    assert summ.n_empty == int((cls == 0).sum())
+    assert summ.visited_area == int(area[cls != 0].sum())
+    if variant == syn.MASK_ROUNDED:
+        assert summ.retained_map == int(area[cls == 1].sum())
+    else:
+        assert summ.retained_map == summ.retained_exact
+    # CSR of visited tiles
+    row_ptr = u32(A["row_ptr"]).astype(np.int64)
+    cols = u32(A["cols"])
+    for qt in (qts if not full else range(A["nq"])):
+        seg = cols[row_ptr[qt]: row_ptr[qt + 1]]
+        kts = np.nonzero(cls[qt])[0]
+        assert np.array_equal(seg & 0x3FFFFFFF, kts)
+        assert np.array_equal(seg >> 30, cls[qt, kts])
+    # execution lists and scheduler order (derived from the map, which matched the oracle)
+    ents, cnts = expected_pair_entries(cls, N, bq, bk)
+    pptr = u32(A["pair_ptr"]).astype(np.int64)
+    pent = u32(A["pair_ent"])
+    pcnt = u32(A["pair_cnt"]).reshape(-1, 2)
+    for p in range(A["npairs"]):
+        assert np.array_equal(pent[pptr[p]: pptr[p + 1]], ents[p]), p
+        assert tuple(pcnt[p]) == cnts[p]
+    work = pcnt.sum(axis=1).astype(np.int64)
+    order = u32(A["pair_order"]).astype(np.int64)
+    assert np.array_equal(np.sort(order), np.arange(A["npairs"]))
+    assert np.array_equal(order, np.lexsort((np.arange(len(work)), -work)))
+    assert summ.pair_entries == sum(len(e) for e in ents)
+    assert summ.pair_half_tiles == int(work.sum())
+    return summ
+
+
+TINY_MAPS = [(r, lay, var, bq, bk) for r in (0, 1) for lay in (0, 1) for var in (0, 1)
+             for (bq, bk) in ((64, 64), (128, 64), (256, 128))]
+
+
+@pytest.mark.parametrize("route,layout,variant,bq,bk", TINY_MAPS)
+def test_tilemap_tiny(S, route, layout, variant, bq, bk):
+    w = syn.TINY.replace(layout=layout)
+    check_tilemap(S, w, route, variant, bq, bk)
+
+
+@pytest.mark.parametrize("route,variant,bq,bk", [(0, 0, 128, 128), (1, 0, 128, 128), (1, 1, 64, 64),
+                                                  (0, 1, 512, 128), (1, 0, 256, 64)])
+def test_tilemap_medium_ragged(S, route, variant, bq, bk):
+    w = syn.Workload("m2", frames=6, grid_h=13, grid_w=17, routes=(route,), d=128, frame_window=2,
+                     spatial_band=9, sink_frames=1)
+    check_tilemap(S, w, route, variant, bq, bk)
+    check_tilemap(S, w.replace(sink_frames=2, layout=1), route, variant, bq, bk)
+
+
+@pytest.mark.parametrize("route,variant,bq,bk", [(0, 0, 128, 128), (1, 0, 128, 128), (0, 1, 256, 64),
+                                                  (1, 1, 512, 128)])
+def test_tilemap_pages_shape(S, route, variant, bq, bk):
+    w = syn.MIXED_75K
+    nq = -(-w.tokens // bq)
+    qts = sorted({0, 1, 2, 27, 28, 29, nq // 3, nq // 2, nq - 3, nq - 2, nq - 1})
+    summ = check_tilemap(S, w, route, variant, bq, bk, qts=qts)
+    assert summ.retained_exact == (1969920000 if route == 0 else 2220817200)
+
+
+def test_tilemap_1440p_totals(S):
+    w = syn.P1440
+    for route in (0, 1):
+        nq = -(-w.tokens // 128)
+        check_tilemap(S, w, route, 0, 128, 128, qts=[0, 113, nq // 2, nq - 1])
+
+
+# ------------------------------------------------------------------------------ permutation
+@pytest.mark.parametrize("w", [syn.TINY, MEDIUM, syn.MIXED_75K, MEDIUM.replace(layout=1, sink_frames=2)],
+                         ids=lambda w: f"{w.name}-L{w.layout}-F{w.sink_frames}")
+def test_permute_matches_oracle(S, w):
+    g, m, _ = gp.geom_mask_tile(w)
+    x = torch.randn(w.heads, w.tokens, w.d, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
+    xd = x.cuda()
+    y = torch.empty_like(xd)
+    S.svg_permute(xd, y, w.routes, g, m)
+    z = torch.empty_like(xd)
+    S.svg_permute(y, z, w.routes, g, m, inverse=True)
+    torch.cuda.synchronize()
+    yc = y.cpu()
+    for h, r in enumerate(w.routes):
+        pi = oracle.perm_table(r, w.layout, w.frames, w.frame_size, w.sink_frames)
+        exp = torch.empty_like(x[h])
+        exp[torch.as_tensor(pi)] = x[h]
+        assert torch.equal(yc[h].view(torch.int16), exp.view(torch.int16))
+    assert torch.equal(z.cpu().view(torch.int16), x.view(torch.int16))
+
+
+# ------------------------------------------------------------------------------ attention
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("variant", [0, 1])
+def test_attention_tiny(S, mode, variant):
+    w = syn.TINY
+    q, k, v = syn.make_qkv(w)
+    out, lse, st = gp.run_path(w, q, k, v, mode=mode, variant=variant)
+    assert st == 0
+    gp.compare_rows(w, q, k, v, out, lse, variant=variant)
+
+
+@pytest.mark.parametrize("bq,bk", [(128, 128), (256, 64), (64, 128), (512, 64)])
+@pytest.mark.parametrize("variant", [0, 1])
+def test_attention_medium_ragged(S, bq, bk, variant):
+    w = MEDIUM
+    q, k, v = syn.make_qkv(w, seed_offset=3)
+    out, lse, st = gp.run_path(w, q, k, v, variant=variant, bq=bq, bk=bk)
+    assert st == 0
+    gp.compare_rows(w, q, k, v, out, lse, variant=variant, bq=bq, bk=bk)
+
+
+@pytest.mark.parametrize("d,bk", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_dense_matches_oracle(S, d, bk):
+    w = MEDIUM.replace(d=d, bk=bk)
+    q, k, v = syn.make_qkv(w, seed_offset=5)
+    out, lse, st = gp.run_path(w, q, k, v, dense=True, bk=bk)
+    assert st == 0
+    gp.compare_rows(w, q, k, v, out, lse, all_kept=True)
+
+
+EDGE = [
+    syn.Workload("one_token", frames=1, grid_h=1, grid_w=1, routes=(0,), d=64, frame_window=0, spatial_band=0),
+    syn.Workload("one_frame_ragged", frames=1, grid_h=7, grid_w=11, routes=(0, 1), d=128, frame_window=0,
+                 spatial_band=3),
+    syn.Workload("no_sink", frames=4, grid_h=6, grid_w=9, routes=(0, 1), d=128, frame_window=1, spatial_band=4,
+                 sink_frames=0),
+    syn.Workload("zero_window", frames=5, grid_h=6, grid_w=9, routes=(0, 1), d=64, frame_window=0,
+                 spatial_band=0, bq=64, bk=64),
+    syn.Workload("full_space_major", frames=6, grid_h=8, grid_w=10, routes=(1, 0, 1), d=128, frame_window=1,
+                 spatial_band=5, layout=1),
+    syn.Workload("two_sink_frames", frames=7, grid_h=5, grid_w=9, routes=(1, 0), d=128, frame_window=1,
+                 spatial_band=3, sink_frames=2, bq=256, bk=64),
+    syn.Workload("window_covers_all", frames=3, grid_h=9, grid_w=13, routes=(0,), d=128, frame_window=5,
+                 spatial_band=0),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
+@pytest.mark.parametrize("variant", [0, 1])
+def test_attention_edge_cases(S, w, variant):
+    q, k, v = syn.make_qkv(w, seed_offset=11)
+    for mode in (0, 1):
+        out, lse, st = gp.run_path(w, q, k, v, mode=mode, variant=variant)
+        assert st == 0
+        gp.compare_rows(w, q, k, v, out, lse, variant=variant)
+
+
+def test_rounded_row_without_keys_gives_zero(S):
+    # band 0 over a wide frame: most temporal tiles are far below half full, so rounding
+    # drops every tile of some rows; those rows must come out as O = 0, LSE = -inf.
+    w = syn.Workload("sparse_rounded", frames=3, grid_h=16, grid_w=32, routes=(1,), d=64, frame_window=0,
+                     spatial_band=0, sink_frames=0, variant=1, bq=128, bk=128)
+    q, k, v = syn.make_qkv(w, seed_offset=2)
+    out, lse, st = gp.run_path(w, q, k, v)
+    assert st == 0
+    stats = gp.compare_rows(w, q, k, v, out, lse, variant=1)
+    assert not torch.isfinite(lse).all()  # some rows really had no key
+    assert stats
+
+
+def test_naive_equals_split_up_to_rounding(S):
+    w = MEDIUM
+    q, k, v = syn.make_qkv(w, seed_offset=7)
+    a, la, _ = gp.run_path(w, q, k, v, mode=0)
+    b, lb, _ = gp.run_path(w, q, k, v, mode=1)
+    diff = (a.float() - b.float()).abs().max().item()
+    assert diff <= 4e-3 and torch.allclose(la, lb, atol=1e-4, rtol=0)
+
+
+# --- the pages' sizes: sampled rows (seeded) plus every row of the ragged last tile
+def _pages(w, rows=512, variant=None, bq=None, bk=None, mode=0):
+    q, k, v = syn.make_qkv(w)
+    out, lse, st = gp.run_path(w, q, k, v, variant=variant, bq=bq, bk=bk, mode=mode)
+    assert st == 0
+
+    def rows_of(h):
+        r = syn.sample_rows(w.replace(sample_rows=rows), h)
+        return np.unique(np.concatenate([r.numpy(), gp.tail_rows(w, h, 96)]))
+
+    return gp.compare_rows(w, q, k, v, out, lse, rows_per_head=rows_of, variant=variant, bq=bq, bk=bk)
+
+
+def test_attention_pages_spatial(S):
+    _pages(syn.SPATIAL_75K, rows=2048)
+
+
+def test_attention_pages_temporal(S):
+    _pages(syn.TEMPORAL_75K, rows=2048)
+
+
+@pytest.mark.parametrize("bq,bk", syn.TILE_SWEEP)
+@pytest.mark.parametrize("variant", [0, 1])
+def test_attention_pages_mixed_sweep(S, bq, bk, variant):
+    _pages(syn.MIXED_75K, rows=128, variant=variant, bq=bq, bk=bk)
+
+
+def test_attention_pages_mixed_naive(S):
+    _pages(syn.MIXED_75K, rows=256, mode=1)
+
+
+def test_attention_1440p(S):
+    _pages(syn.P1440, rows=256)
