@@ -195,6 +195,9 @@ def main():
     ap.add_argument("--bk", type=int, default=128)
     ap.add_argument("--mode", default="split", choices=["split", "naive"])
     ap.add_argument("--no-extras", action="store_true", help="skip the side measurements")
+    ap.add_argument("--quick", action="store_true",
+                    help="only the timed steps (no side measurements, e2e or CPU baseline): for profiler runs")
+    ap.add_argument("--heads", type=int, default=0, help="use only the first H heads of the workload")
     ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=48, help="oracle rows per head per --impl reference step")
     args = ap.parse_args()
@@ -202,6 +205,8 @@ def main():
         args.warmup = 3
     world, rank, local = dist_env()
     w = syn.WORKLOADS[args.workload].replace(bq=args.bq, bk=args.bk)
+    if args.heads > 0:
+        w = w.replace(routes=w.routes[: args.heads])
 
     if args.impl == "reference":
         return run_reference(args, w, world, rank)
@@ -286,16 +291,18 @@ def main():
                 "peak_kind": f"{peak_kind} bf16 burst"}
 
     extras = {}
-    if not args.no_extras:
+    if not (args.no_extras or args.quick):
         extras = side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws, summ, P, stream,
                                    dev)
 
     # ---------------------------------------------------------------- end to end through host buffers
-    e2e = end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream,
-                     args)
+    e2e = None
+    if not args.quick:
+        e2e = end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream,
+                         args)
 
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.quick:
         sec, nrows, nthreads = oracle_sample(w, q_cpu, k_cpu, v_cpu, args.cpu_rows)
         full = sec * (w.tokens * w.heads) / nrows
         cpu = {"value": eff_flop / full / 1e12, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
