@@ -187,6 +187,38 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
 
 }  // namespace
 
+
+// ---------------------------------------------------------------------------------------
+// Scratch of svg_attention_fwd_noalloc: a file-scope device array, so that callers that
+// cannot allocate need not pass one. In host code `g_noalloc_scratch` only names the
+// symbol; its device address comes from cudaGetSymbolAddress, looked up once per device
+// (with that device current) on the first call there.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SVG_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void* noalloc_scratch(int* rc) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *rc = SVG_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      *rc = SVG_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
 extern "C" {
 
 int svg_version(void) { return 10000; }
@@ -295,6 +327,20 @@ int svg_dense_attention_fwd(const void* q, const void* k, const void* v, void* o
                             int32_t* d_status, void* stream) {
   return run_attention(q, k, v, o, lse, heads, tokens, d, scale, nullptr, nullptr, nullptr, nullptr, nullptr, 0, bk,
                        SVG_MODE_SPLIT, true, d_scratch, scratch_bytes, d_status, static_cast<cudaStream_t>(stream));
+}
+
+int svg_attention_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,
+                              int64_t tokens, int32_t d, float scale, const uint8_t* h_route,
+                              const void* d_ws_spatial, const void* d_ws_temporal, svg_geom geom, svg_mask mask,
+                              svg_tile tile, int32_t mode, int32_t* d_status, void* stream) {
+  if (svg_attention_scratch_bytes() > SVG_NOALLOC_SCRATCH_BYTES) return SVG_ERR_ARG;
+  int rc = check_qkvo(q, k, v, o, lse, heads, tokens, d);  // reject bad arguments before any CUDA call
+  if (rc) return rc;
+  void* scratch = noalloc_scratch(&rc);
+  if (!scratch) return rc;
+  return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
+                       tile.bq, tile.bk, mode, false, scratch, SVG_NOALLOC_SCRATCH_BYTES, d_status,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int svg_read_status(const void* d_scratch_or_status, int32_t* h_status, void* stream) {

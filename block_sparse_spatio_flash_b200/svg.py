@@ -73,6 +73,8 @@ _sig = {
     "svg_dense_attention_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _i32,
                                                _vp, _sz, _vp, _vp]),
     "svg_read_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int32), _vp]),
+    "svg_attention_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p,
+                                                 _vp, _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -183,6 +185,18 @@ def svg_dense_attention_fwd(q, k, v, o, bk=128, scratch=None, lse=None, scale: f
     _check(_lib.svg_dense_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), heads, tokens, d, scale,
                                         bk, _ptr(scratch), scratch.numel() * scratch.element_size(), _ptr(status),
                                         _stream(stream)), "svg_dense_attention_fwd")
+    return o
+
+
+def svg_attention_fwd_noalloc(q, k, v, o, routes, ws_spatial, ws_temporal, geom, mask, tile,
+                              mode=SVG_MODE_SPLIT, lse=None, scale: float = 0.0, status=None,
+                              stream=None) -> torch.Tensor:
+    """svg_attention_fwd without a scratch argument: the library's static device scratch is
+    used instead (shared by every call on the device; overlapping calls race)."""
+    heads, tokens, d = q.shape
+    _check(_lib.svg_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), heads, tokens, d, scale,
+                                          _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile,
+                                          mode, _ptr(status), _stream(stream)), "svg_attention_fwd_noalloc")
     return o
 
 

@@ -174,6 +174,34 @@ int svg_dense_attention_fwd(const void *q, const void *k, const void *v, void *o
                             void *d_scratch, size_t scratch_bytes, int32_t *d_status,
                             void *stream);
 
+/*
+ * Allocation-free variant of svg_attention_fwd. The paper has no counterpart; it exists for
+ * callers that cannot allocate device memory themselves, e.g. a plugin inside a host
+ * framework that hands it only the input and output buffers, or a server that forbids
+ * device allocation after start-up because cudaMalloc may synchronise the device and
+ * fragment a fixed memory budget.
+ * Instead of a caller-provided scratch buffer it uses a static device array of
+ * SVG_NOALLOC_SCRATCH_BYTES bytes inside the library (every device that loads the library
+ * holds it until the process exits). Arguments are those of svg_attention_fwd without
+ * d_scratch / scratch_bytes.
+ *   - The first call on each device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and clears it on `stream` before its
+ *     kernel runs; calls that overlap on the GPU (other streams, other host threads) race on
+ *     it and must be serialised by the caller.
+ *   - d_status (nullable) receives the device status as in svg_attention_fwd; without it,
+ *     device-side errors are written only to the shared array and cannot be read back.
+ *   - Returns SVG_ERR_ARG when the scratch the call needs exceeds SVG_NOALLOC_SCRATCH_BYTES
+ *     (it needs svg_attention_scratch_bytes(), independent of the problem size), plus every
+ *     error svg_attention_fwd returns. Allocates nothing (no cudaMalloc / cudaFree).
+ */
+#define SVG_NOALLOC_SCRATCH_BYTES 256
+int svg_attention_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                              int32_t heads, int64_t tokens, int32_t d, float scale,
+                              const uint8_t *h_route, const void *d_ws_spatial,
+                              const void *d_ws_temporal, svg_geom geom, svg_mask mask,
+                              svg_tile tile, int32_t mode, int32_t *d_status, void *stream);
+
 /* Reads the device status word of a scratch buffer (or d_status). Synchronises `stream`. */
 int svg_read_status(const void *d_scratch_or_status, int32_t *h_status, void *stream);
 
