@@ -5,6 +5,7 @@
 // Nothing here allocates device memory.
 #include <math.h>
 #include <mutex>
+#include <stdio.h>
 #include <string.h>
 
 #include "svg_common.cuh"
@@ -18,9 +19,15 @@ int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t 
 
 using namespace svg;
 
+namespace svg {
+int record_cuda_error(const char* what, int cuda_error);
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+thread_local char g_last_error[192] = "none";
 
 // Compute capability and SM count of the current device (cached per device).
 int device_info(int* num_sms) {
@@ -28,14 +35,16 @@ int device_info(int* num_sms) {
   static int sms[kMaxDevices] = {0};
   static int ok[kMaxDevices] = {0};  // 0 unknown, 1 sm_100, -1 other
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SVG_ERR_CUDA;
+  cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return record_cuda_error("cudaGetDevice", ge);
+  if (dev < 0 || dev >= kMaxDevices) return SVG_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(mu);
   if (ok[dev] == 0) {
     int major = 0, minor = 0, n = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return SVG_ERR_CUDA;
+    cudaError_t e1 = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e1 == cudaSuccess) e1 = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e1 == cudaSuccess) e1 = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e1 != cudaSuccess) return record_cuda_error("cudaDeviceGetAttribute", e1);
     ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
     sms[dev] = n;
   }
@@ -83,7 +92,7 @@ EncodeTiledFn encode_fn() {
 // (128 bytes, one swizzle atom wide) x box_rows rows x 1 head; rows past the end read 0.
 int encode_qkv_map(CUtensorMap* m, const void* base, int heads, int tokens, int d, int box_rows) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return SVG_ERR_CUDA;
+  if (!fn) return record_cuda_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", (int)cudaErrorSymbolNotFound);
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)tokens, (cuuint64_t)heads};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)tokens * d * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
@@ -91,7 +100,11 @@ int encode_qkv_map(CUtensorMap* m, const void* base, int heads, int tokens, int 
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? SVG_OK : SVG_ERR_CUDA;
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled: CUresult %d", (int)r);
+    return SVG_ERR_CUDA;
+  }
+  return SVG_OK;
 }
 
 int check_qkvo(const void* q, const void* k, const void* v, const void* o, const float* lse, int heads,
@@ -179,8 +192,9 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
   if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, bk))) return rc;
   if ((rc = encode_qkv_map(&P.tm_v, v, heads, N, d, bk))) return rc;
-  if (cudaMemsetAsync(scratch, 0, kScratchBytes, st) != cudaSuccess) return SVG_ERR_CUDA;
-  if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int32_t), st) != cudaSuccess) return SVG_ERR_CUDA;
+  cudaError_t me = cudaMemsetAsync(scratch, 0, kScratchBytes, st);
+  if (me == cudaSuccess && d_status) me = cudaMemsetAsync(d_status, 0, sizeof(int32_t), st);
+  if (me != cudaSuccess) return record_cuda_error("cudaMemsetAsync(scratch)", me);
   const int grid = (int)(P.n_items < num_sms ? P.n_items : num_sms);
   return launch_attention(P, d, bk, grid, st);
 }
@@ -208,8 +222,9 @@ void* noalloc_scratch(int* rc) {
   std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-      *rc = SVG_ERR_CUDA;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      *rc = record_cuda_error("cudaGetSymbolAddress", e);
       return nullptr;
     }
     addr[dev] = p;
@@ -219,7 +234,15 @@ void* noalloc_scratch(int* rc) {
 
 }  // namespace
 
+int svg::record_cuda_error(const char* what, int cuda_error) {
+  const cudaError_t e = static_cast<cudaError_t>(cuda_error);
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", what, cudaGetErrorString(e), cuda_error);
+  return SVG_ERR_CUDA;
+}
+
 extern "C" {
+
+const char* svg_last_cuda_error(void) { return g_last_error; }
 
 int svg_version(void) { return 10000; }
 
@@ -277,8 +300,10 @@ int svg_tilemap_summary(const void* d_ws, svg_tilemap_summary_t* h_out, void* st
   if (!d_ws || !h_out || !aligned(d_ws, 256)) return SVG_ERR_ARG;
   TmHeader h;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(&h, d_ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SVG_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SVG_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(&h, d_ws, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return record_cuda_error("cudaMemcpyAsync(summary)", e);
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return record_cuda_error("cudaStreamSynchronize(summary)", e);
   if (h.magic != kTmMagic) return SVG_ERR_WORKSPACE;
   h_out->retained_exact = h.retained_exact;
   h_out->retained_map = h.retained_map;
@@ -346,9 +371,10 @@ int svg_attention_fwd_noalloc(const void* q, const void* k, const void* v, void*
 int svg_read_status(const void* d_scratch_or_status, int32_t* h_status, void* stream) {
   if (!d_scratch_or_status || !h_status || !aligned(d_scratch_or_status, 4)) return SVG_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(h_status, d_scratch_or_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return SVG_ERR_CUDA;
-  return cudaStreamSynchronize(st) == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(h_status, d_scratch_or_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return record_cuda_error("cudaMemcpyAsync(status)", e);
+  e = cudaStreamSynchronize(st);
+  return e == cudaSuccess ? SVG_OK : record_cuda_error("cudaStreamSynchronize(status)", e);
 }
 
 }  // extern "C"

@@ -49,7 +49,6 @@ struct Cfg {
   static constexpr uint32_t kPCol = BK / 2;
   __host__ __device__ static constexpr uint32_t o_col(int h) { return 256u + (uint32_t)D * h; }
   static_assert(kStages >= 2, "ring too small");
-  static_assert((2 * kStages + 31) * 8 <= 1024, "control block");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -58,31 +57,62 @@ struct ItemInfo {
   const uint32_t* ents;
 };
 
+// Shared-memory control block, addressed by 32-bit shared addresses so that the roles keep
+// a single base register instead of one generic pointer per barrier.
+//   [0, NS)        kv_full[s]    TMA K/V tile landed in ring slot s
+//   [NS, 2NS)      kv_empty[s]   MMAs done reading ring slot s
+//   2NS + 0 / 1    q_full / q_free
+//   2NS + 2 + h    s_full[h]     S_h = Q_h K^T (and every earlier MMA) complete
+//   2NS + 4 + h    p_ready[h]    P_h in TMEM, O_h corrected (128 arrivals)
+//   2NS + 6 + h    o_done[h]     last P V of half h complete
+//   2NS + 8 + h    o_free[h]     epilogue finished reading O_h (128 arrivals)
+//   2NS + 10 + i   item_full[i]  work item published in slot i
+//   2NS + 12 + i   item_empty[i] slot i read by the MMA warp and the 8 softmax warps
+//   2NS + 14       drain         final MMA completion
+//   2NS + 16 ...   two ItemInfo slots, TMEM base, abort flag, workspace check
+template <int NS>
 struct Ctl {
-  uint64_t* kv_full;
-  uint64_t* kv_empty;
-  uint64_t *q_full, *q_free, *s_full, *p_ready, *o_done, *o_free, *item_full, *item_empty, *drain;
-  ItemInfo* items;
-  volatile int* abort_flag;
+  uint32_t base;  // shared address of the control block
   int* status;
+  __device__ __forceinline__ uint32_t kv_full(uint32_t s) const { return base + 8u * s; }
+  __device__ __forceinline__ uint32_t kv_empty(uint32_t s) const { return base + 8u * (NS + s); }
+  __device__ __forceinline__ uint32_t q_full() const { return base + 8u * (2 * NS + 0); }
+  __device__ __forceinline__ uint32_t q_free() const { return base + 8u * (2 * NS + 1); }
+  __device__ __forceinline__ uint32_t s_full(int h) const { return base + 8u * (2 * NS + 2 + h); }
+  __device__ __forceinline__ uint32_t p_ready(int h) const { return base + 8u * (2 * NS + 4 + h); }
+  __device__ __forceinline__ uint32_t o_done(int h) const { return base + 8u * (2 * NS + 6 + h); }
+  __device__ __forceinline__ uint32_t o_free(int h) const { return base + 8u * (2 * NS + 8 + h); }
+  __device__ __forceinline__ uint32_t item_full(uint32_t i) const { return base + 8u * (2 * NS + 10 + i); }
+  __device__ __forceinline__ uint32_t item_empty(uint32_t i) const { return base + 8u * (2 * NS + 12 + i); }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * (2 * NS + 14); }
+  static constexpr uint32_t kItemsOff = 8u * (2 * NS + 16);  // 2 x 40 bytes
+  static constexpr uint32_t kTmemOff = kItemsOff + 96;
+  static constexpr uint32_t kAbortOff = kTmemOff + 8;
+  static constexpr uint32_t kBadWsOff = kAbortOff + 8;
+  static constexpr uint32_t kBytes = kBadWsOff + 8;
 };
 
-__device__ __forceinline__ void raise_error(const Ctl& c, int code) {
-  *c.abort_flag = 1;
-  atomicCAS(c.status, 0, code);
+__device__ __forceinline__ int ld_shared_volatile(uint32_t addr) {
+  int v;
+  asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared(uint32_t addr, int v) {
+  asm volatile("st.volatile.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // Bounded wait on an mbarrier phase. Returns false on timeout or when another role aborted.
-__device__ __noinline__ bool wait_bar(const Ctl& c, uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+// abort_addr: shared address of the abort flag; status: global status word.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t abort_addr, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0) {
-      if (*c.abort_flag) return false;
+      if (ld_shared_volatile(abort_addr)) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        raise_error(c, SVG_ERR_TIMEOUT);
+        st_shared(abort_addr, 1);
+        atomicCAS(status, 0, SVG_ERR_TIMEOUT);
         return false;
       }
     }
@@ -90,8 +120,7 @@ __device__ __noinline__ bool wait_bar(const Ctl& c, uint64_t* bar, uint32_t pari
 }
 
 // Drain wait: ignores the abort flag, short limit; used only on the error path.
-__device__ __noinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
+__device__ __noinline__ void drain_bar(uint32_t a, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(a, parity))
     if (globaltimer_ns() - t0 > 200000000ull) return;
@@ -147,6 +176,29 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+// 2^x on the FMA / integer pipes, to take part of the exponentials off the MUFU unit.
+// Cody-Waite style range reduction: n = round(x) (by the 1.5*2^23 rounding trick), f = x - n in
+// [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
+// error on [-1/2, 1/2] (fitted by linear programming, max rel. error 7.5e-5, far below the bf16
+// rounding of P); 2^n is added to the exponent field. Exact 0 for x < -125 (masked scores).
+constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f, kExpC2 = 2.426111251e-01f,
+                kExpC3 = 5.517166853e-02f;
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.f);
+  const float r = xc + 12582912.f;  // 1.5 * 2^23: n sits in the low mantissa bits of r
+  const float n = r - 12582912.f;
+  const float f = xc - n;
+  const float p = fmaf(fmaf(fmaf(kExpC3, f, kExpC2), f, kExpC1), f, kExpC0);
+  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
+  return x < -125.f ? 0.f : y;
+}
+
+// Columns (mod 8) whose exponential is computed by exp2_poly instead of ex2.approx.
+#ifndef SVG_POLY_MASK
+#define SVG_POLY_MASK 0x00u
+#endif
+constexpr uint32_t kPolyMask = SVG_POLY_MASK;
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low 16 bits)
   return *reinterpret_cast<uint32_t*>(&v);
@@ -156,54 +208,41 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
   using C = Cfg<D, BK>;
+  constexpr int NS = C::kStages;
+  using K = Ctl<NS>;
+  static_assert(K::kBytes <= 1024, "control block");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  uint8_t* sQ = smem;
-  uint8_t* sRing = smem + C::kQBytes;
-  uint8_t* ctl_base = smem + C::kDataBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ctl_base);
-  Ctl c;
-  c.kv_full = bars;
-  c.kv_empty = bars + C::kStages;
-  uint64_t* b = bars + 2 * C::kStages;
-  c.q_full = b + 0;
-  c.q_free = b + 1;
-  c.s_full = b + 2;      // [2]
-  c.p_ready = b + 4;     // [2]
-  c.o_done = b + 6;      // [2]
-  c.o_free = b + 8;      // [2]
-  c.item_full = b + 10;  // [2]
-  c.item_empty = b + 12; // [2]
-  c.drain = b + 14;
-  static_assert(sizeof(ItemInfo) == 40, "item slot size");
-  c.items = reinterpret_cast<ItemInfo*>(b + 16);            // 2 x 40 bytes: b[16..26)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b + 28);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(b + 29);
-  int* bad_ws = reinterpret_cast<int*>(b + 30);
-  c.abort_flag = abort_flag;
+  const uint32_t sbase = raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sQ = sbase, sRing = sbase + C::kQBytes;
+  K c;
+  c.base = sbase + C::kDataBytes;
   c.status = P.status;
-
+  uint8_t* ctl_gen = smem_raw + (c.base - raw);  // generic pointer to the control block
+  ItemInfo* items = reinterpret_cast<ItemInfo*>(ctl_gen + K::kItemsOff);
+  const uint32_t abort_addr = c.base + K::kAbortOff;
+  int* status = P.status;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(c.kv_full + s, 1);
-      mbar_init(c.kv_empty + s, 1);
+    for (int st = 0; st < NS; ++st) {
+      mbar_init(reinterpret_cast<uint64_t*>(ctl_gen) + st, 1);       // kv_full
+      mbar_init(reinterpret_cast<uint64_t*>(ctl_gen) + NS + st, 1);  // kv_empty
     }
-    mbar_init(c.q_full, 1);
-    mbar_init(c.q_free, 1);
+    uint64_t* b = reinterpret_cast<uint64_t*>(ctl_gen) + 2 * NS;
+    mbar_init(b + 0, 1);  // q_full
+    mbar_init(b + 1, 1);  // q_free
     for (int h = 0; h < 2; ++h) {
-      mbar_init(c.s_full + h, 1);
-      mbar_init(c.p_ready + h, 128);
-      mbar_init(c.o_done + h, 1);
-      mbar_init(c.o_free + h, 128);
-      mbar_init(c.item_full + h, 1);
-      mbar_init(c.item_empty + h, 9);
+      mbar_init(b + 2 + h, 1);     // s_full
+      mbar_init(b + 4 + h, 128);   // p_ready
+      mbar_init(b + 6 + h, 1);     // o_done
+      mbar_init(b + 8 + h, 128);   // o_free
+      mbar_init(b + 10 + h, 1);    // item_full
+      mbar_init(b + 12 + h, 9);    // item_empty
     }
-    mbar_init(c.drain, 1);
-    *abort_flag = 0;
+    mbar_init(b + 14, 1);  // drain
+    *reinterpret_cast<volatile int*>(ctl_gen + K::kAbortOff) = 0;
     // the tile maps must have been built for exactly these parameters
     int bad = 0;
     if (!P.dense) {
@@ -216,12 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                h->bk != P.exp_bk || h->nk != P.nk || h->npairs != P.npairs;
       }
     }
-    *bad_ws = bad;
+    *reinterpret_cast<int*>(ctl_gen + K::kBadWsOff) = bad;
     if (bad) atomicCAS(P.status, 0, SVG_ERR_WORKSPACE);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(reinterpret_cast<uint32_t*>(ctl_gen + K::kTmemOff), 512);
     tmem_relinquish();
   }
   if (warp == kProducerWarp && lane == 0) {
@@ -232,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const bool skip_all = *bad_ws != 0;
+  const uint32_t tmem = *reinterpret_cast<uint32_t*>(ctl_gen + K::kTmemOff);
+  const bool skip_all = *reinterpret_cast<int*>(ctl_gen + K::kBadWsOff) != 0;
 
   if (!skip_all && warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
@@ -242,21 +281,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       bool q_issued = false;
       for (uint32_t it = 0;; ++it) {
         const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
-        if (!wait_bar(c, c.item_empty + slot, ph ^ 1u)) break;
+        if (!wait_bar(c.item_empty(slot), ph ^ 1u, abort_addr, status)) break;
         const uint32_t idx = atomicAdd(P.counter, 1u);
         const ItemInfo inf = decode_item<BK>(P, idx);
-        c.items[slot] = inf;
-        mbar_arrive(c.item_full + slot);
+        items[slot] = inf;
+        mbar_arrive(c.item_full(slot));
         if (!inf.valid) break;
         if (inf.nA + inf.nB > 0) {
-          if (!wait_bar(c, c.q_free, (q_iter & 1u) ^ 1u)) break;
+          if (!wait_bar(c.q_free(), (q_iter & 1u) ^ 1u, abort_addr, status)) break;
           ++q_iter;
           const uint32_t bytes = (uint32_t)C::kQHalfBytes * ((inf.nA > 0) + (inf.nB > 0));
-          mbar_expect_tx(c.q_full, bytes);
+          mbar_expect_tx(c.q_full(), bytes);
           for (int h = 0; h < 2; ++h) {
             if ((h == 0 ? inf.nA : inf.nB) == 0) continue;
             for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_3d(sQ + h * C::kQHalfBytes + ch * (128 * 128), &P.tm_q, c.q_full, ch * 64,
+              tma_load_3d(sQ + h * C::kQHalfBytes + ch * (128 * 128), &P.tm_q, c.q_full(), ch * 64,
                           inf.pair * kPairRows + h * kHalfRows, inf.head);
           }
           q_issued = true;
@@ -266,28 +305,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           const uint32_t ent = get_entry<BK>(P, inf, e);
           const int row0 = (int)ent_kt(ent) * BK;
           for (int w = 0; w < 2; ++w) {
-            const uint32_t s = kv_pos % C::kStages, phs = (kv_pos / C::kStages) & 1u;
-            if (!wait_bar(c, c.kv_empty + s, phs ^ 1u)) {
+            const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
+            if (!wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status)) {
               ok = false;
               break;
             }
-            mbar_expect_tx(c.kv_full + s, C::kTileBytes);
-            uint8_t* dst = sRing + s * C::kTileBytes;
+            mbar_expect_tx(c.kv_full(st), C::kTileBytes);
+            const uint32_t dst = sRing + st * C::kTileBytes;
             for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_3d(dst + ch * (BK * 128), w == 0 ? &P.tm_k : &P.tm_v, c.kv_full + s, ch * 64, row0,
+              tma_load_3d(dst + ch * (BK * 128), w == 0 ? &P.tm_k : &P.tm_v, c.kv_full(st), ch * 64, row0,
                           inf.head);
             ++kv_pos;
           }
         }
         if (!ok) break;
       }
-      if (*abort_flag) {  // let issued copies land before the CTA may exit
-        const uint32_t n = kv_pos < (uint32_t)C::kStages ? kv_pos : (uint32_t)C::kStages;
+      if (ld_shared_volatile(abort_addr)) {  // let issued copies land before the CTA may exit
+        const uint32_t n = kv_pos < (uint32_t)NS ? kv_pos : (uint32_t)NS;
         for (uint32_t i = 0; i < n; ++i) {
           const uint32_t pos = kv_pos - 1 - i;
-          drain_bar(c.kv_full + pos % C::kStages, (pos / C::kStages) & 1u);
+          drain_bar(c.kv_full(pos % NS), (pos / NS) & 1u);
         }
-        if (q_issued) drain_bar(c.q_full, (q_iter - 1) & 1u);
+        if (q_issued) drain_bar(c.q_full(), (q_iter - 1) & 1u);
       }
     }
     __syncwarp();
@@ -296,92 +335,96 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(BK, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(D, true);
-      const uint32_t q_base = smem_u32(sQ), ring_base = smem_u32(sRing);
-      uint32_t kv_pos = 0, q_iter = 0, p_cnt[2] = {0, 0}, of_cnt[2] = {0, 0};
+      // Descriptors are built once; per k-step and per ring slot only the start-address
+      // field (bits [0,14), address >> 4) moves, and no address exceeds 256 KB, so a plain add
+      // on the low word never carries out of the field.
+      const uint64_t qdesc = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t kdesc = smem_desc_sw128(sRing, 16, 1024);
+      const uint64_t vdesc = smem_desc_sw128(sRing, BK * 128, 1024);
+      uint32_t kv_pos = 0, q_iter = 0, p_cnt0 = 0, p_cnt1 = 0, of_cnt0 = 0, of_cnt1 = 0;
       bool ok = true;
       for (uint32_t it = 0; ok; ++it) {
         const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
-        if (!wait_bar(c, c.item_full + slot, ph)) break;
-        const ItemInfo inf = c.items[slot];
-        mbar_arrive(c.item_empty + slot);
+        if (!wait_bar(c.item_full(slot), ph, abort_addr, status)) break;
+        const ItemInfo inf = items[slot];
+        mbar_arrive(c.item_empty(slot));
         if (!inf.valid) break;
-        const bool has_q = inf.nA + inf.nB > 0;
-        if (has_q) {
-          if (!wait_bar(c, c.q_full, q_iter & 1u)) break;
+        if (inf.nA + inf.nB > 0) {
+          if (!wait_bar(c.q_full(), q_iter & 1u, abort_addr, status)) break;
           ++q_iter;
           tc_fence_after();
         }
-        int remaining[2] = {inf.nA, inf.nB};
-        bool prev_act[2] = {false, false}, has_o[2] = {false, false};
+        int rem0 = inf.nA, rem1 = inf.nB;   // active entries left per half
+        uint32_t prev_act = 0, has_o = 0;    // bit h: half h active at the previous entry / O_h written
         uint32_t prev_v = 0;
-        // O_h += P_h V(prev): waits for P and (first time) for the epilogue to free O_h.
-        auto issue_pv = [&](int h, uint32_t vpos) -> bool {
-          if (!wait_bar(c, c.p_ready + h, p_cnt[h] & 1u)) return false;
-          ++p_cnt[h];
-          if (!has_o[h]) {
-            if (!wait_bar(c, c.o_free + h, (of_cnt[h] & 1u) ^ 1u)) return false;
-            ++of_cnt[h];
-          }
-          if (!wait_bar(c, c.kv_full + vpos % C::kStages, (vpos / C::kStages) & 1u)) return false;
-          tc_fence_after();
-          const uint32_t vaddr = ring_base + (vpos % C::kStages) * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(vaddr + kk * 2048, BK * 128, 1024);
-            umma_ts(tmem + C::o_col(h), tmem + C::s_col(h) + C::kPCol + kk * 8, bdesc, idesc_o,
-                    (has_o[h] || kk > 0) ? 1u : 0u);
-          }
-          has_o[h] = true;
-          if (--remaining[h] == 0) umma_commit(c.o_done + h);
-          return true;
-        };
-        for (int e = 0; e < inf.count; ++e) {
-          const uint32_t ent = get_entry<BK>(P, inf, e);
+        for (int e = 0; e <= inf.count && ok; ++e) {
+          // entry e (or, at e == count, only the trailing P V of the last entry)
+          const bool last = e == inf.count;
+          const uint32_t ent = last ? 0u : get_entry<BK>(P, inf, e);
           const uint32_t kpos = kv_pos, vpos = kv_pos + 1;
-          kv_pos += 2;
-          if (!wait_bar(c, c.kv_full + kpos % C::kStages, (kpos / C::kStages) & 1u)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t kaddr = ring_base + (kpos % C::kStages) * C::kTileBytes;
-          for (int h = 0; h < 2 && ok; ++h) {
-            if (prev_act[h] && !issue_pv(h, prev_v)) {
-              ok = false;
-              break;
+          bool k_ready = false;
+          const uint64_t kd = kdesc + (((kpos % NS) * C::kTileBytes) >> 4);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (!ok) break;
+            if ((prev_act >> h) & 1u) {  // O_h += P_h V(e-1): needs P_h and, first time, a free O_h
+              uint32_t& pc = h == 0 ? p_cnt0 : p_cnt1;
+              uint32_t& oc = h == 0 ? of_cnt0 : of_cnt1;
+              ok = wait_bar(c.p_ready(h), pc & 1u, abort_addr, status);
+              ++pc;
+              if (ok && !((has_o >> h) & 1u)) {
+                ok = wait_bar(c.o_free(h), (oc & 1u) ^ 1u, abort_addr, status);
+                ++oc;
+              }
+              if (ok) ok = wait_bar(c.kv_full(prev_v % NS), (prev_v / NS) & 1u, abort_addr, status);
+              if (!ok) break;
+              tc_fence_after();
+              const uint64_t vd = vdesc + (((prev_v % NS) * C::kTileBytes) >> 4);
+              const uint32_t acc0 = (has_o >> h) & 1u;
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma_ts(tmem + C::o_col(h), tmem + C::s_col(h) + C::kPCol + kk * 8, vd + ((kk * 2048) >> 4),
+                        idesc_o, (acc0 || kk > 0) ? 1u : 0u);
+              has_o |= 1u << h;
+              int& rem = h == 0 ? rem0 : rem1;
+              if (--rem == 0) umma_commit(c.o_done(h));
             }
-            const bool act = ent_flag(ent, h) != kFlagSkip;
+            const bool act = !last && ent_flag(ent, h) != kFlagSkip;
             if (act) {
-              const uint32_t qaddr = q_base + h * C::kQHalfBytes;
+              if (!k_ready) {
+                ok = wait_bar(c.kv_full(kpos % NS), (kpos / NS) & 1u, abort_addr, status);
+                if (!ok) break;
+                tc_fence_after();
+                k_ready = true;
+              }
+              const uint64_t qd = qdesc + ((h * C::kQHalfBytes) >> 4);
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 bytes along K inside the swizzle atom
-                const uint64_t adesc = smem_desc_sw128(qaddr + (kk >> 2) * (128 * 128) + off, 16, 1024);
-                const uint64_t bdesc = smem_desc_sw128(kaddr + (kk >> 2) * (BK * 128) + off, 16, 1024);
-                umma_ss(tmem + C::s_col(h), adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                // 16 bf16 = 32 bytes along K inside a 128-byte swizzle atom; 64 columns per atom
+                const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
+                umma_ss(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
               }
-              umma_commit(c.s_full + h);
+              umma_commit(c.s_full(h));
             }
-            prev_act[h] = act;
+            prev_act = (prev_act & ~(1u << h)) | ((act ? 1u : 0u) << h);
           }
           if (!ok) break;
-          umma_commit(c.kv_empty + kpos % C::kStages);               // K(e) read by the S MMAs
-          if (e > 0) umma_commit(c.kv_empty + (vpos - 2) % C::kStages);  // V(e-1) read by the PVs
-          if (e == inf.count - 1) umma_commit(c.q_free);              // Q read by the last S MMA
-          prev_v = vpos;
-        }
-        if (!ok) break;
-        for (int h = 0; h < 2; ++h)
-          if (prev_act[h] && !issue_pv(h, prev_v)) {
-            ok = false;
-            break;
+          if (e > 0) umma_commit(c.kv_empty(prev_v % NS));  // V(e-1) read by the P V MMAs
+          if (last) break;
+          if (!k_ready) {  // (an entry always has an active half; never release a slot still loading)
+            ok = wait_bar(c.kv_full(kpos % NS), (kpos / NS) & 1u, abort_addr, status);
+            if (!ok) break;
           }
-        if (!ok) break;
-        if (inf.count > 0) umma_commit(c.kv_empty + prev_v % C::kStages);
+          umma_commit(c.kv_empty(kpos % NS));            // K(e) read by the S MMAs
+          if (e == inf.count - 1) umma_commit(c.q_free());  // Q read by the last S MMA
+          prev_v = vpos;
+          kv_pos += 2;
+        }
       }
       // all issued MMAs complete before TMEM is released
-      umma_commit(c.drain);
-      drain_bar(c.drain, 0);
+      umma_commit(c.drain());
+      drain_bar(c.drain(), 0);
     }
     __syncwarp();
   } else if (!skip_all && warp < 8) {
@@ -396,39 +439,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     uint32_t s_cnt = 0, od_cnt = 0;
     for (uint32_t it = 0;; ++it) {
       const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
-      if (!__all_sync(0xffffffffu, wait_bar(c, c.item_full + slot, ph))) break;  // warp-uniform exit
-      const ItemInfo inf = c.items[slot];
+      if (!__all_sync(0xffffffffu, wait_bar(c.item_full(slot), ph, abort_addr, status))) break;
+      const ItemInfo inf = items[slot];
       __syncwarp();
-      if (lane == 0) mbar_arrive(c.item_empty + slot);
+      if (lane == 0) mbar_arrive(c.item_empty(slot));
       if (!inf.valid) break;
       const int row = inf.pair * kPairRows + h * kHalfRows + lr;
       const bool in_range = row < P.N;
       const int nmine = h == 0 ? inf.nA : inf.nB;
-      __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + (in_range ? row : 0)) * D;
       if (nmine == 0) {  // no kept key for any row of this half (rounded masks only)
         if (in_range) {
-          uint4 z = make_uint4(0, 0, 0, 0);
+          __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + row) * D;
+          const uint4 z = make_uint4(0, 0, 0, 0);
           for (int x = 0; x < D / 8; ++x) reinterpret_cast<uint4*>(orow)[x] = z;
           if (P.lse) P.lse[(size_t)inf.head * P.N + row] = -INFINITY;
         }
         continue;
       }
-      const MaskGeom& g = P.g[inf.cls];
       const int prow = in_range ? row : P.N - 1;
-      int lo = 0, hi = 0;
-      if (!P.dense) row_interval(g, prow, lo, hi);
-      const int se = P.dense ? 0 : sink_end(g);
-      const bool per = !P.dense && periodic_sink(g);
-      const uint8_t* rcls = P.cls[inf.cls] + (size_t)(prow / (P.bq > 0 ? P.bq : 1)) * P.nk;
+      // kept keys of this row: [0, se) U [lo, hi) U (periodic sink), see svg_common.cuh
+      int lo = 0, hi = 0, se = 0;
+      bool per = false;
+      if (!P.dense) {
+        const MaskGeom& g = P.g[inf.cls];
+        row_interval(g, prow, lo, hi);
+        se = sink_end(g);
+        per = periodic_sink(g);
+      }
       float m = -INFINITY, l = 0.f;
       bool first = true;
       bool ok = true;
+      uint32_t ent_next = inf.count > 0 ? get_entry<BK>(P, inf, 0) : 0u;
       for (int e = 0; e < inf.count; ++e) {
-        const uint32_t ent = get_entry<BK>(P, inf, e);
+        const uint32_t ent = ent_next;
+        if (e + 1 < inf.count) ent_next = get_entry<BK>(P, inf, e + 1);  // hide the load latency
         const uint32_t f = ent_flag(ent, h);
         if (f == kFlagSkip) continue;
         const int c0 = (int)ent_kt(ent) * BK;
-        if (!__all_sync(0xffffffffu, wait_bar(c, c.s_full + h, s_cnt & 1u))) {
+        if (!__all_sync(0xffffffffu, wait_bar(c.s_full(h), s_cnt & 1u, abort_addr, status))) {
           ok = false;
           break;
         }
@@ -441,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
         for (int q = 0; q < BK / 32; ++q) tmem_ld_fence32(r + q * 32);
         float* s = reinterpret_cast<float*>(r);
-        // ---- masking
+        // ---- masking (boundary tiles, ragged key tail, naive mode)
         const bool elem = (f == kFlagMasked) || (P.naive && !P.dense);
         if (elem || f == kFlagBounds) {
           const int nn = P.N - c0;
@@ -450,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             for (int j = 0; j < BK; ++j)
               if (j >= nn) s[j] = -INFINITY;
           } else if (P.variant == SVG_MASK_ROUNDED) {
+            const uint8_t* rcls = P.cls[inf.cls] + (size_t)(prow / P.bq) * P.nk;
             const bool rowkept = __ldg(rcls + ent_kt(ent)) == 1;
 #pragma unroll
             for (int j = 0; j < BK; ++j)
@@ -465,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 if (!keep) s[j] = -INFINITY;
               }
             } else {
+              const MaskGeom& g = P.g[inf.cls];
               int rr = c0 % g.T;
 #pragma unroll
               for (int j = 0; j < BK; ++j) {
@@ -475,53 +525,64 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             }
           }
         }
-        // ---- online softmax
-        float mx = s[0];
+        // ---- online softmax: row max and row sum as independent chains
+        float mx4[4];
 #pragma unroll
-        for (int j = 1; j < BK; ++j) mx = fmaxf(mx, s[j]);
+        for (int i = 0; i < 4; ++i) mx4[i] = s[i];
+#pragma unroll
+        for (int j = 4; j < BK; j += 4)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(mx4[i], s[j + i]);
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         const float m_new = fmaxf(m, mx);
         const bool need = (m_new > m) && (m == -INFINITY || (m_new - m) * sl2 > kRescaleThreshold);
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = (m_new == -INFINITY) ? 1.f : ex2f((m - m_new) * sl2);
-          if (!first) {
-#pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
-              uint32_t o[32];
-              tmem_ld32(tO + q * 32, o);
-              tmem_ld_wait();
-              tmem_ld_fence32(o);
-#pragma unroll
-              for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-              tmem_st32(tO + q * 32, o);
-            }
-          }
+        // the O correction itself runs after P is stored, when the score row is dead
+        const bool rescale = __any_sync(0xffffffffu, need);
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = (m_new == -INFINITY) ? 1.f : ex2f((m - m_new) * sl2);
           l *= alpha;
           m = m_new;
         }
         const float base = (m == -INFINITY) ? 0.f : m * sl2;
-        uint32_t pk[BK / 2];
-        float lsum = 0.f;
+        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < BK; j += 2) {
-          const float p0 = ex2f(fmaf(s[j], sl2, -base));
-          const float p1 = ex2f(fmaf(s[j + 1], sl2, -base));
-          lsum += p0 + p1;
-          pk[j / 2] = pack_bf16(p0, p1);
+          const float x0 = fmaf(s[j], sl2, -base);
+          const float x1 = fmaf(s[j + 1], sl2, -base);
+          const float p0 = ((kPolyMask >> (j & 7)) & 1u) ? exp2_poly(x0) : ex2f(x0);
+          const float p1 = ((kPolyMask >> ((j + 1) & 7)) & 1u) ? exp2_poly(x1) : ex2f(x1);
+          ls4[j & 3] += p0;
+          ls4[(j + 1) & 3] += p1;
+          r[j / 2] = pack_bf16(p0, p1);  // packed P overwrites the consumed front of the row
         }
-        l += lsum;
+        l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
 #pragma unroll
-        for (int q = 0; q < BK / 64; ++q) tmem_st32(tP + q * 32, pk + q * 32);
+        for (int q = 0; q < BK / 64; ++q) tmem_st32(tP + q * 32, r + q * 32);
+        if (rescale && !first) {  // O_h holds every earlier P V (S_h's commit covered them)
+#pragma unroll 1
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
+            tmem_ld_wait();
+            tmem_ld_fence32(o);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(tO + q * 32, o);
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(c.p_ready + h);
+        mbar_arrive(c.p_ready(h));
         first = false;
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16
-      if (!__all_sync(0xffffffffu, wait_bar(c, c.o_done + h, od_cnt & 1u))) break;
+      if (!__all_sync(0xffffffffu, wait_bar(c.o_done(h), od_cnt & 1u, abort_addr, status))) break;
       ++od_cnt;
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + prow) * D;
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
         uint32_t o[32];
@@ -542,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
       }
       tc_fence_before();
-      mbar_arrive(c.o_free + h);
+      mbar_arrive(c.o_free(h));
       if (in_range && P.lse)
         P.lse[(size_t)inf.head * P.N + row] =
             l > 0.f ? (m * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -560,10 +621,11 @@ template <int D, int BK>
 static int launch_t(const AttnParams& P, int grid, cudaStream_t st) {
   using C = Cfg<D, BK>;
   auto kern = attn_kernel<D, BK>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-    return SVG_ERR_CUDA;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return record_cuda_error("cudaFuncSetAttribute(attn_kernel)", e);
   kern<<<grid, kThreads, C::kSmemBytes, st>>>(P);
-  return cudaGetLastError() == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SVG_OK : record_cuda_error("launch attn_kernel", e);
 }
 
 int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st) {

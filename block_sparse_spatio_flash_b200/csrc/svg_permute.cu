@@ -83,7 +83,8 @@ int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const
   if (bx > need) bx = need;
   if (bx < 1) bx = 1;
   permute_kernel<<<dim3((unsigned)bx, (unsigned)heads), 512, 0, st>>>(P);
-  return cudaGetLastError() == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SVG_OK : record_cuda_error("launch permute_kernel", e);
 }
 
 }  // namespace svg

@@ -266,14 +266,16 @@ int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* 
   P.pair_ent = reinterpret_cast<uint32_t*>(base + L.pair_ent);
   P.pair_cnt = reinterpret_cast<uint32_t*>(base + L.pair_cnt);
   P.pair_order = reinterpret_cast<uint32_t*>(base + L.pair_order);
-  if (cudaMemsetAsync(base, 0, 256, st) != cudaSuccess) return SVG_ERR_CUDA;
+  cudaError_t e = cudaMemsetAsync(base, 0, 256, st);
+  if (e != cudaSuccess) return record_cuda_error("cudaMemsetAsync(tile-map header)", e);
   tm_classify<<<L.nq, 256, 0, st>>>(P, geom, mask, tile, route);
   tm_pair_count<<<L.npairs, 256, 0, st>>>(P);
   tm_scan<<<1, 1024, 0, st>>>(P);
   tm_fill_cols<<<L.nq, 256, 0, st>>>(P);
   tm_fill_pairs<<<L.npairs, 256, 0, st>>>(P);
   tm_sort_pairs<<<(L.npairs + 127) / 128, 128, 0, st>>>(P);
-  return cudaGetLastError() == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SVG_OK : record_cuda_error("launch tile-map kernels", e);
 }
 
 }  // namespace svg

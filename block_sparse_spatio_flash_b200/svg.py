@@ -62,6 +62,7 @@ _u8p = ctypes.POINTER(ctypes.c_uint8)
 _sig = {
     "svg_version": (ctypes.c_int, []),
     "svg_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "svg_last_cuda_error": (ctypes.c_char_p, []),
     "svg_tilemap_bytes": (_sz, [svg_geom, svg_tile]),
     "svg_tilemap_get_layout": (ctypes.c_int, [svg_geom, svg_tile, ctypes.POINTER(svg_tilemap_layout)]),
     "svg_build_tilemap": (ctypes.c_int, [svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp]),
@@ -84,7 +85,8 @@ for _name, (_res, _args) in _sig.items():
 class SvgError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {svg_error_string(code)} (code {code})")
+        detail = f"; last CUDA error: {svg_last_cuda_error()}" if code == SVG_ERR_CUDA else ""
+        super().__init__(f"{where}: {svg_error_string(code)} (code {code}){detail}")
 
 
 def _check(code: int, where: str) -> int:
@@ -133,6 +135,10 @@ def svg_version() -> int:
 
 def svg_error_string(code: int) -> str:
     return _lib.svg_error_string(code).decode()
+
+
+def svg_last_cuda_error() -> str:
+    return _lib.svg_last_cuda_error().decode()
 
 
 def svg_tilemap_bytes(geom: svg_geom, tile: svg_tile) -> int:

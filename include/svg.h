@@ -208,6 +208,10 @@ int svg_read_status(const void *d_scratch_or_status, int32_t *h_status, void *st
 /* Static description of an error code. */
 const char *svg_error_string(int code);
 
+/* Which CUDA call last failed on the calling thread and why (after an SVG_ERR_CUDA return);
+ * "none" if none has. The string stays valid until the next failing call on that thread. */
+const char *svg_last_cuda_error(void);
+
 /* Library version (major*10000 + minor*100 + patch). */
 int svg_version(void);
 
