@@ -105,6 +105,23 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
 
 
+def aggregate_over_ranks(local_ms: float, local_flop: float, world: int, device=None):
+    """Step time of the job = max over ranks (device-timed); value = all ranks' FLOP over it.
+
+    Every rank calls this at the same point (it is a collective when world > 1)."""
+    ms = float(local_ms)
+    flop = float(local_flop)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms, flop], dtype=torch.float64, device=device)
+        tmax = t[:1].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        tsum = t[1:].clone()
+        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+        ms, flop = float(tmax.item()), float(tsum.item())
+    return ms, flop / (ms * 1e-3) / 1e12
+
+
 def time_events(fn, iters, stream):
     """Mean ms per call over `iters` calls, CUDA events on the launching stream."""
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -270,16 +287,10 @@ def main():
         if world > 1:
             dist.barrier()
     per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    ms = total_ms / args.steps
+    ms, value = aggregate_over_ranks(ev[0].elapsed_time(ev[-1]) / args.steps, eff_flop, world, dev)
     status = S.svg_read_status(scratch)
     if status != 0:
         raise RuntimeError(f"device status {status}: {S.svg_error_string(status)}")
-    value = world * eff_flop / (ms * 1e-3) / 1e12
     clocks = clk.summary()
 
     # ---------------------------------------------------------------- roofline of the attention kernel
@@ -412,15 +423,10 @@ def end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, ef
     for _ in range(2):
         e2e_step()
     n = max(3, min(20, args.steps // 5))
-    ms = time_events(e2e_step, n, stream)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms, value = aggregate_over_ranks(time_events(e2e_step, n, stream), eff_flop, world, dev)
     h2d = 3 * q_cpu.numel() * 2
     d2h = q_cpu.numel() * 2
-    return {"value": world * eff_flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+    return {"value": value, "unit": "TFLOP/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n}
 
 

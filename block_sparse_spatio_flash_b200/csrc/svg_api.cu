@@ -5,6 +5,7 @@
 // Nothing here allocates device memory.
 #include <math.h>
 #include <mutex>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -15,6 +16,7 @@ int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* 
 int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const uint8_t* h_route, svg_geom geom,
                    svg_mask mask, int inverse, int num_sms, cudaStream_t st);
 int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st);
+int launch_attention_pair(const AttnParams& P, int bk, int max_clusters, cudaStream_t st);
 }  // namespace svg
 
 using namespace svg;
@@ -107,6 +109,17 @@ int encode_qkv_map(CUtensorMap* m, const void* base, int heads, int tokens, int 
   return SVG_OK;
 }
 
+// The single-SM kernel serves every call; SVG_KERNEL=pair in the environment (read once)
+// selects the SM-pair kernel (two-SM MMAs, each SM loading half of every K/V tile) for d = 128,
+// to compare the two.
+bool use_pair_kernel(int d) {
+  static const bool pair = [] {
+    const char* v = getenv("SVG_KERNEL");
+    return v && strcmp(v, "pair") == 0;
+  }();
+  return d == 128 && pair;
+}
+
 int check_qkvo(const void* q, const void* k, const void* v, const void* o, const float* lse, int heads,
                int64_t tokens, int d) {
   if (!q || !k || !v || !o) return SVG_ERR_ARG;
@@ -135,16 +148,19 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   std::lock_guard<std::mutex> lock(mu);
   memset(&P, 0, sizeof(P));
   const int N = (int)tokens;
+  const bool pair = use_pair_kernel(d);
   P.H = heads;
   P.N = N;
   P.nk = (N + bk - 1) / bk;
   P.npairs = (N + kPairRows - 1) / kPairRows;
-  const int64_t items = (int64_t)heads * P.npairs;
+  P.nquads = (N + kQuadRows - 1) / kQuadRows;
+  const int64_t items = (int64_t)heads * (pair ? P.nquads : P.npairs);
   if (items > 0x7FFFFFFF) return SVG_ERR_ARG;
   P.n_items = (int)items;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   P.sl2 = sc * 1.4426950408889634f;
   P.dense = dense ? 1 : 0;
+  P.bkm = bk;
   P.naive = mode == SVG_MODE_NAIVE ? 1 : 0;
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
@@ -175,6 +191,10 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
       P.pair_ent[c] = reinterpret_cast<const uint32_t*>(b + L.pair_ent);
       P.pair_cnt[c] = reinterpret_cast<const uint32_t*>(b + L.pair_cnt);
       P.pair_order[c] = reinterpret_cast<const uint32_t*>(b + L.pair_order);
+      P.quad_ptr[c] = reinterpret_cast<const uint32_t*>(b + L.quad_ptr);
+      P.quad_ent[c] = reinterpret_cast<const uint32_t*>(b + L.quad_ent);
+      P.quad_cnt[c] = reinterpret_cast<const uint32_t*>(b + L.quad_cnt);
+      P.quad_order[c] = reinterpret_cast<const uint32_t*>(b + L.quad_order);
     }
     P.variant = mask->variant;
     P.bq = bq;
@@ -189,12 +209,15 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
     P.exp_bq = bq;
     P.exp_bk = bk;
   }
+  // TMA boxes: Q 128 rows; one-SM kernel K and V bk rows; SM-pair kernel: each SM loads bk/2
+  // keys of K (all 128 dims) and all bk keys of V for 64 of the dims.
   if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
-  if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, bk))) return rc;
+  if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, pair ? bk / 2 : bk))) return rc;
   if ((rc = encode_qkv_map(&P.tm_v, v, heads, N, d, bk))) return rc;
   cudaError_t me = cudaMemsetAsync(scratch, 0, kScratchBytes, st);
   if (me == cudaSuccess && d_status) me = cudaMemsetAsync(d_status, 0, sizeof(int32_t), st);
   if (me != cudaSuccess) return record_cuda_error("cudaMemsetAsync(scratch)", me);
+  if (pair) return launch_attention_pair(P, bk, (int)(P.n_items < num_sms / 2 ? P.n_items : num_sms / 2), st);
   const int grid = (int)(P.n_items < num_sms ? P.n_items : num_sms);
   return launch_attention(P, d, bk, grid, st);
 }
@@ -277,10 +300,14 @@ int svg_tilemap_get_layout(svg_geom geom, svg_tile tile, svg_tilemap_layout* out
   out->pair_ent = L.pair_ent;
   out->pair_cnt = L.pair_cnt;
   out->pair_order = L.pair_order;
+  out->quad_ptr = L.quad_ptr;
+  out->quad_ent = L.quad_ent;
+  out->quad_cnt = L.quad_cnt;
+  out->quad_order = L.quad_order;
   out->nq = L.nq;
   out->nk = L.nk;
   out->npairs = L.npairs;
-  out->reserved = 0;
+  out->nquads = L.nquads;
   return SVG_OK;
 }
 
@@ -313,6 +340,8 @@ int svg_tilemap_summary(const void* d_ws, svg_tilemap_summary_t* h_out, void* st
   h_out->visited_area = h.visited_area;
   h_out->pair_entries = h.pair_entries;
   h_out->pair_half_tiles = h.pair_half_tiles;
+  h_out->quad_entries = h.quad_entries;
+  h_out->quad_phase_tiles = h.quad_phase_tiles;
   return SVG_OK;
 }
 

@@ -103,7 +103,7 @@ __device__ __forceinline__ void st_shared(uint32_t addr, int v) {
 
 // Bounded wait on an mbarrier phase. Returns false on timeout or when another role aborted.
 // abort_addr: shared address of the abort flag; status: global status word.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t abort_addr, int* status) {
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -117,6 +117,11 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t ab
       }
     }
   }
+}
+
+// Fast path inline (an already-completed phase costs one try_wait), the bounded loop out of line.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t abort_addr, int* status) {
+  return mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, abort_addr, status);
 }
 
 // Drain wait: ignores the abort flag, short limit; used only on the error path.
@@ -168,40 +173,6 @@ __device__ ItemInfo decode_item(const AttnParams& P, uint32_t idx) {
     it.nB = (int)__ldg(P.pair_cnt[c] + 2 * it.pair + 1);
   }
   return it;
-}
-
-__device__ __forceinline__ float ex2f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 2^x on the FMA / integer pipes, to take part of the exponentials off the MUFU unit.
-// Cody-Waite style range reduction: n = round(x) (by the 1.5*2^23 rounding trick), f = x - n in
-// [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
-// error on [-1/2, 1/2] (fitted by linear programming, max rel. error 7.5e-5, far below the bf16
-// rounding of P); 2^n is added to the exponent field. Exact 0 for x < -125 (masked scores).
-constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f, kExpC2 = 2.426111251e-01f,
-                kExpC3 = 5.517166853e-02f;
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float r = xc + 12582912.f;  // 1.5 * 2^23: n sits in the low mantissa bits of r
-  const float n = r - 12582912.f;
-  const float f = xc - n;
-  const float p = fmaf(fmaf(fmaf(kExpC3, f, kExpC2), f, kExpC1), f, kExpC0);
-  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
-  return x < -125.f ? 0.f : y;
-}
-
-// Columns (mod 8) whose exponential is computed by exp2_poly instead of ex2.approx.
-#ifndef SVG_POLY_MASK
-#define SVG_POLY_MASK 0x00u
-#endif
-constexpr uint32_t kPolyMask = SVG_POLY_MASK;
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low 16 bits)
-  return *reinterpret_cast<uint32_t*>(&v);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -349,10 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const ItemInfo inf = items[slot];
         mbar_arrive(c.item_empty(slot));
         if (!inf.valid) break;
-        if (inf.nA + inf.nB > 0) {
+        if (inf.nA + inf.nB > 0) {  // (TMA data: the barrier alone orders it for the tensor core)
           if (!wait_bar(c.q_full(), q_iter & 1u, abort_addr, status)) break;
           ++q_iter;
-          tc_fence_after();
         }
         int rem0 = inf.nA, rem1 = inf.nB;   // active entries left per half
         uint32_t prev_act = 0, has_o = 0;    // bit h: half h active at the previous entry / O_h written
@@ -391,10 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             }
             const bool act = !last && ent_flag(ent, h) != kFlagSkip;
             if (act) {
-              if (!k_ready) {
+              if (!k_ready) {  // TMA data: no tcgen05 fence needed; S_h's order against the softmax's
+                               // TMEM reads comes from the fence after the last P_h wait
                 ok = wait_bar(c.kv_full(kpos % NS), (kpos / NS) & 1u, abort_addr, status);
                 if (!ok) break;
-                tc_fence_after();
                 k_ready = true;
               }
               const uint64_t qd = qdesc + ((h * C::kQHalfBytes) >> 4);

@@ -23,7 +23,8 @@ namespace svg {
 constexpr uint32_t kTmMagic = 0x53564731u;  // "SVG1"
 constexpr int kMaxHeads = 4096;
 constexpr int64_t kMaxTokens = 1 << 22;
-constexpr int kPairRows = 256;  // query rows per execution item: two 128-row halves
+constexpr int kPairRows = 256;  // query rows per item of the one-SM kernel: two 128-row halves
+constexpr int kQuadRows = 512;  // query rows per item of the two-SM kernel: 2 SMs x two halves
 constexpr int kHalfRows = 128;
 
 // ---------------------------------------------------------------------------------------
@@ -140,15 +141,16 @@ __host__ __device__ inline int row_kept_in(const MaskGeom& g, int lo, int hi, in
 // Tile-map workspace record (offset 0 of the workspace, 256 bytes).
 struct TmHeader {
   uint32_t magic, version;
-  int32_t T, H, W, route, k, b, F0, variant, layout, bq, bk, nq, nk, npairs, N, pad0;
+  int32_t T, H, W, route, k, b, F0, variant, layout, bq, bk, nq, nk, npairs, N, nquads;
   unsigned long long retained_exact, retained_map, n_full, n_boundary, n_empty, visited_area,
-      pair_entries, pair_half_tiles;
+      pair_entries, pair_half_tiles, quad_entries, quad_phase_tiles;
 };
 static_assert(sizeof(TmHeader) <= 256, "header must fit in 256 bytes");
 
 struct TmLayout {
   uint64_t total, cls, cnt, row_ptr, cols, pair_ptr, pair_ent, pair_cnt, pair_order;
-  int nq, nk, npairs;
+  uint64_t quad_ptr, quad_ent, quad_cnt, quad_order;
+  int nq, nk, npairs, nquads;
 };
 
 // Records a failed CUDA call (what + error) for svg_last_cuda_error; returns SVG_ERR_CUDA.
@@ -171,14 +173,25 @@ inline TmLayout tm_layout(int64_t N, int bq, int bk) {
   L.pair_ent = off;   off = align_up(off + 4 * (uint64_t)L.npairs * L.nk, 256);
   L.pair_cnt = off;   off = align_up(off + 8 * (uint64_t)L.npairs, 256);
   L.pair_order = off; off = align_up(off + 4 * (uint64_t)L.npairs, 256);
+  L.nquads = (int)((N + kQuadRows - 1) / kQuadRows);
+  L.quad_ptr = off;   off = align_up(off + 4 * (uint64_t)(L.nquads + 1), 256);
+  L.quad_ent = off;   off = align_up(off + 4 * (uint64_t)L.nquads * L.nk, 256);
+  L.quad_cnt = off;   off = align_up(off + 8 * (uint64_t)L.nquads, 256);
+  L.quad_order = off; off = align_up(off + 4 * (uint64_t)L.nquads, 256);
   L.total = off;
   return L;
 }
 
-// Execution-list entry: kt | flagA << 28 | flagB << 30.
+// Execution-list entry of a group of G 128-row blocks (G = 2: pair, G = 4: quad):
+// kt in the low (32 - 2G) bits, then one 2-bit flag per block, block i at bit 32 - 2G + 2i.
+// In a quad, block i = 2 * rank + half (rank = SM of the pair, half = MMA phase).
 enum : uint32_t { kFlagSkip = 0, kFlagFull = 1, kFlagMasked = 2, kFlagBounds = 3 };
 __host__ __device__ inline uint32_t ent_kt(uint32_t e) { return e & 0x0FFFFFFFu; }
 __host__ __device__ inline uint32_t ent_flag(uint32_t e, int half) { return (e >> (28 + 2 * half)) & 3u; }
+__host__ __device__ inline uint32_t qent_kt(uint32_t e) { return e & 0x00FFFFFFu; }
+__host__ __device__ inline uint32_t qent_flag(uint32_t e, int rank, int half) {
+  return (e >> (24 + 4 * rank + 2 * half)) & 3u;
+}
 
 // Scratch of the attention entry points: [0] status, [1] reserved, [2] work counter.
 constexpr size_t kScratchBytes = 256;
@@ -191,6 +204,7 @@ struct AttnParams {
   int H, N, npairs, nk, n_items;
   float sl2;  // scale * log2(e)
   int dense, naive, variant, bq;
+  int bkm;  // key-tile width of the entries (tile map's bk, or the dense call's bk)
   MaskGeom g[2];
   const TmHeader* hdr[2];
   const uint8_t* cls[2];
@@ -198,6 +212,11 @@ struct AttnParams {
   const uint32_t* pair_ent[2];
   const uint32_t* pair_cnt[2];
   const uint32_t* pair_order[2];
+  const uint32_t* quad_ptr[2];
+  const uint32_t* quad_ent[2];
+  const uint32_t* quad_cnt[2];
+  const uint32_t* quad_order[2];
+  int nquads;
   int uses[2];
   int exp_T, exp_H, exp_W, exp_k, exp_b, exp_F0, exp_variant, exp_layout, exp_bq, exp_bk;
   int* status;
@@ -366,15 +385,129 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, M = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n, bool b_mn_major) {
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, M = 128 (one SM) or 256 (SM pair).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n, bool b_mn_major, int m = 128) {
   return (1u << 4)                      // D format fp32
          | (1u << 7)                    // A format bf16
          | (1u << 10)                   // B format bf16
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(n >> 3) << 17)   // N / 8
-         | ((uint32_t)(128 >> 4) << 24);  // M / 16
+         | ((uint32_t)(m >> 4) << 24);  // M / 16
 }
+
+// ---- CTA pairs (clusters of 2) and the two-SM tensor-core forms ----
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared::cluster address of the variable at shared address `a` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive (release, cluster scope) on an mbarrier given by its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t a) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an mbarrier of either
+// CTA of the pair (bar = shared::cluster address). No multicast.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                                 int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A B over both SMs of the pair: each SM supplies 128 rows of A and half of B's N columns
+// (same shared-memory offsets in both), and receives its 128 rows of D in its own TMEM.
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The mbarrier (shared::cluster address, in either CTA) arrives once all pair MMAs issued so
+// far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// ---- softmax arithmetic shared by the attention kernels ----
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA / integer pipes, to take part of the exponentials off the MUFU unit.
+// Cody-Waite style range reduction: n = round(x) (by the 1.5*2^23 rounding trick), f = x - n in
+// [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
+// error on [-1/2, 1/2] (fitted by linear programming, max rel. error 7.5e-5, far below the bf16
+// rounding of P); 2^n is added to the exponent field. Exact 0 for x < -125 (masked scores).
+constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f, kExpC2 = 2.426111251e-01f,
+                kExpC3 = 5.517166853e-02f;
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.f);
+  const float r = xc + 12582912.f;  // 1.5 * 2^23: n sits in the low mantissa bits of r
+  const float n = r - 12582912.f;
+  const float f = xc - n;
+  const float p = fmaf(fmaf(fmaf(kExpC3, f, kExpC2), f, kExpC1), f, kExpC0);
+  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
+  return x < -125.f ? 0.f : y;
+}
+
+// Columns (mod 8) whose exponential is computed by exp2_poly instead of ex2.approx.
+#ifndef SVG_POLY_MASK
+#define SVG_POLY_MASK 0x00u
+#endif
+constexpr uint32_t kPolyMask = SVG_POLY_MASK;
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low 16 bits)
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 #endif  // __CUDACC__
 
 }  // namespace svg

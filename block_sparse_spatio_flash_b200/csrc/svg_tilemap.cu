@@ -14,6 +14,17 @@
 
 namespace svg {
 
+// Execution lists of groups of G 128-row blocks (pairs: G = 2, quads: G = 4).
+struct GroupLists {
+  uint32_t* ptr;    // [ngroups + 1]
+  uint32_t* ent;    // [ngroups * nk]
+  uint32_t* cnt;    // [2 * ngroups]: entries in which MMA phase h (block index % 2) is active
+  uint32_t* order;  // [ngroups] by descending work
+  int ngroups;
+  unsigned long long* tot_entries;
+  unsigned long long* tot_phase_tiles;
+};
+
 struct TmParams {
   MaskGeom g;
   int bq, bk, nq, nk, npairs, variant;
@@ -21,10 +32,7 @@ struct TmParams {
   uint32_t* cnt;
   uint32_t* row_ptr;
   uint32_t* cols;
-  uint32_t* pair_ptr;
-  uint32_t* pair_ent;
-  uint32_t* pair_cnt;
-  uint32_t* pair_order;
+  GroupLists pairs, quads;
   TmHeader* hdr;
 };
 
@@ -61,7 +69,7 @@ __global__ void __launch_bounds__(256) tm_classify(TmParams P, svg_geom geom, sv
     h->T = geom.frames; h->H = geom.grid_h; h->W = geom.grid_w; h->route = route;
     h->k = mask.frame_window; h->b = mask.spatial_band; h->F0 = mask.sink_frames;
     h->variant = mask.variant; h->layout = mask.layout; h->bq = tile.bq; h->bk = tile.bk;
-    h->nq = P.nq; h->nk = P.nk; h->npairs = P.npairs; h->N = g.N;
+    h->nq = P.nq; h->nk = P.nk; h->npairs = P.npairs; h->N = g.N; h->nquads = P.quads.ngroups;
   }
   __syncthreads();
   unsigned long long kept_tot = 0, map_tot = 0, nfull = 0, nbnd = 0, nemp = 0, varea = 0;
@@ -109,9 +117,9 @@ __global__ void __launch_bounds__(256) tm_classify(TmParams P, svg_geom geom, sv
   if (threadIdx.x == 0) atomicAdd(&P.hdr->visited_area, s);
 }
 
-// Flag of one 128-row half for k-tile kt, combining the classes of the q-tiles it overlaps.
-__device__ __forceinline__ uint32_t half_flag(const TmParams& P, int pair, int half, int kt) {
-  const int r0 = pair * kPairRows + half * kHalfRows;
+// Flag of the 128-row block starting at row r0 for k-tile kt, combining the classes of the
+// q-tiles it overlaps.
+__device__ __forceinline__ uint32_t block_flag(const TmParams& P, int r0, int kt) {
   if (r0 >= P.g.N) return kFlagSkip;
   const int r1 = min(P.g.N, r0 + kHalfRows);
   const int qa = r0 / P.bq, qb = (r1 - 1) / P.bq;
@@ -127,30 +135,46 @@ __device__ __forceinline__ uint32_t half_flag(const TmParams& P, int pair, int h
   return ragged ? kFlagBounds : kFlagFull;
 }
 
-// One block per 256-row pair: entries, per-half active counts.
-__global__ void __launch_bounds__(256) tm_pair_count(TmParams P) {
+// Entry of group g for k-tile kt (0xFFFFFFFF when no block of the group visits the tile).
+template <int G>
+__device__ __forceinline__ uint32_t group_entry(const TmParams& P, int g, int kt, uint32_t* phase_bits) {
+  uint32_t e = (uint32_t)kt, ph = 0;
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    const uint32_t f = block_flag(P, g * G * kHalfRows + i * kHalfRows, kt);
+    e |= f << (32 - 2 * G + 2 * i);
+    if (f) ph |= 1u << (i & 1);
+  }
+  *phase_bits = ph;
+  return ph ? e : 0xFFFFFFFFu;
+}
+
+// One block per group: number of entries and, per MMA phase, entries where it is active.
+template <int G>
+__global__ void __launch_bounds__(256) tm_group_count(TmParams P, GroupLists L) {
   __shared__ unsigned long long red[8];
-  const int pr = blockIdx.x;
-  uint32_t ne = 0, na = 0, nb = 0;
+  const int g = blockIdx.x;
+  uint32_t ne = 0, n0 = 0, n1 = 0;
   for (int kt = threadIdx.x; kt < P.nk; kt += blockDim.x) {
-    const uint32_t fa = half_flag(P, pr, 0, kt), fb = half_flag(P, pr, 1, kt);
-    ne += (fa | fb) != 0;
-    na += fa != 0;
-    nb += fb != 0;
+    uint32_t ph;
+    const uint32_t e = group_entry<G>(P, g, kt, &ph);
+    ne += e != 0xFFFFFFFFu;
+    n0 += ph & 1u;
+    n1 += (ph >> 1) & 1u;
   }
   unsigned long long s;
   s = block_sum_u64(ne, red);
   if (threadIdx.x == 0) {
-    P.pair_ptr[pr] = (uint32_t)s;
-    atomicAdd(&P.hdr->pair_entries, s);
+    L.ptr[g] = (uint32_t)s;
+    atomicAdd(L.tot_entries, s);
   }
-  s = block_sum_u64(na, red);
-  if (threadIdx.x == 0) P.pair_cnt[2 * pr] = (uint32_t)s;
-  unsigned long long sa = s;
-  s = block_sum_u64(nb, red);
+  s = block_sum_u64(n0, red);
+  if (threadIdx.x == 0) L.cnt[2 * g] = (uint32_t)s;
+  const unsigned long long s0 = s;
+  s = block_sum_u64(n1, red);
   if (threadIdx.x == 0) {
-    P.pair_cnt[2 * pr + 1] = (uint32_t)s;
-    atomicAdd(&P.hdr->pair_half_tiles, sa + s);
+    L.cnt[2 * g + 1] = (uint32_t)s;
+    atomicAdd(L.tot_phase_tiles, s0 + s);
   }
 }
 
@@ -185,7 +209,9 @@ __device__ void block_exclusive_scan(uint32_t* a, int n) {
 __global__ void __launch_bounds__(1024) tm_scan(TmParams P) {
   block_exclusive_scan(P.row_ptr, P.nq);
   __syncthreads();
-  block_exclusive_scan(P.pair_ptr, P.npairs);
+  block_exclusive_scan(P.pairs.ptr, P.pairs.ngroups);
+  __syncthreads();
+  block_exclusive_scan(P.quads.ptr, P.quads.ngroups);
 }
 
 // Ordered compaction of one row of flags, 256 threads, chunk by chunk.
@@ -224,31 +250,33 @@ __global__ void __launch_bounds__(256) tm_fill_cols(TmParams P) {
   });
 }
 
-__global__ void __launch_bounds__(256) tm_fill_pairs(TmParams P) {
-  const int pr = blockIdx.x;
-  compact_row(P.nk, P.pair_ent + P.pair_ptr[pr], [&](int kt) -> uint32_t {
-    const uint32_t fa = half_flag(P, pr, 0, kt), fb = half_flag(P, pr, 1, kt);
-    return (fa | fb) ? ((uint32_t)kt | (fa << 28) | (fb << 30)) : 0xFFFFFFFFu;
+template <int G>
+__global__ void __launch_bounds__(256) tm_fill_groups(TmParams P, GroupLists L) {
+  const int g = blockIdx.x;
+  compact_row(P.nk, L.ent + L.ptr[g], [&](int kt) -> uint32_t {
+    uint32_t ph;
+    return group_entry<G>(P, g, kt, &ph);
   });
 }
 
-// Rank of each pair by (work descending, index ascending); work = active (entry, half)s.
-__global__ void tm_sort_pairs(TmParams P) {
+// Rank of each group by (work descending, index ascending); work = active (entry, phase)s.
+__global__ void tm_sort_groups(GroupLists L) {
   const int p = blockIdx.x * blockDim.x + threadIdx.x;
-  if (p >= P.npairs) return;
-  const uint32_t wp = P.pair_cnt[2 * p] + P.pair_cnt[2 * p + 1];
+  if (p >= L.ngroups) return;
+  const uint32_t wp = L.cnt[2 * p] + L.cnt[2 * p + 1];
   uint32_t rank = 0;
-  for (int q = 0; q < P.npairs; ++q) {
-    const uint32_t wq = P.pair_cnt[2 * q] + P.pair_cnt[2 * q + 1];
+  for (int q = 0; q < L.ngroups; ++q) {
+    const uint32_t wq = L.cnt[2 * q] + L.cnt[2 * q + 1];
     rank += (wq > wp) || (wq == wp && q < p);
   }
-  P.pair_order[rank] = (uint32_t)p;
+  L.order[rank] = (uint32_t)p;
 }
 
 int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* ws, cudaStream_t st) {
   const MaskGeom g = make_geom(geom, mask, route);
   const TmLayout L = tm_layout(g.N, tile.bq, tile.bk);
   uint8_t* base = static_cast<uint8_t*>(ws);
+  auto u32 = [&](uint64_t off) { return reinterpret_cast<uint32_t*>(base + off); };
   TmParams P;
   P.g = g;
   P.bq = tile.bq;
@@ -259,21 +287,24 @@ int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* 
   P.variant = mask.variant;
   P.hdr = reinterpret_cast<TmHeader*>(base);
   P.cls = base + L.cls;
-  P.cnt = reinterpret_cast<uint32_t*>(base + L.cnt);
-  P.row_ptr = reinterpret_cast<uint32_t*>(base + L.row_ptr);
-  P.cols = reinterpret_cast<uint32_t*>(base + L.cols);
-  P.pair_ptr = reinterpret_cast<uint32_t*>(base + L.pair_ptr);
-  P.pair_ent = reinterpret_cast<uint32_t*>(base + L.pair_ent);
-  P.pair_cnt = reinterpret_cast<uint32_t*>(base + L.pair_cnt);
-  P.pair_order = reinterpret_cast<uint32_t*>(base + L.pair_order);
+  P.cnt = u32(L.cnt);
+  P.row_ptr = u32(L.row_ptr);
+  P.cols = u32(L.cols);
+  P.pairs = GroupLists{u32(L.pair_ptr), u32(L.pair_ent), u32(L.pair_cnt), u32(L.pair_order), L.npairs,
+                       &P.hdr->pair_entries, &P.hdr->pair_half_tiles};
+  P.quads = GroupLists{u32(L.quad_ptr), u32(L.quad_ent), u32(L.quad_cnt), u32(L.quad_order), L.nquads,
+                       &P.hdr->quad_entries, &P.hdr->quad_phase_tiles};
   cudaError_t e = cudaMemsetAsync(base, 0, 256, st);
   if (e != cudaSuccess) return record_cuda_error("cudaMemsetAsync(tile-map header)", e);
   tm_classify<<<L.nq, 256, 0, st>>>(P, geom, mask, tile, route);
-  tm_pair_count<<<L.npairs, 256, 0, st>>>(P);
+  tm_group_count<2><<<L.npairs, 256, 0, st>>>(P, P.pairs);
+  tm_group_count<4><<<L.nquads, 256, 0, st>>>(P, P.quads);
   tm_scan<<<1, 1024, 0, st>>>(P);
   tm_fill_cols<<<L.nq, 256, 0, st>>>(P);
-  tm_fill_pairs<<<L.npairs, 256, 0, st>>>(P);
-  tm_sort_pairs<<<(L.npairs + 127) / 128, 128, 0, st>>>(P);
+  tm_fill_groups<2><<<L.npairs, 256, 0, st>>>(P, P.pairs);
+  tm_fill_groups<4><<<L.nquads, 256, 0, st>>>(P, P.quads);
+  tm_sort_groups<<<(L.npairs + 127) / 128, 128, 0, st>>>(P.pairs);
+  tm_sort_groups<<<(L.nquads + 127) / 128, 128, 0, st>>>(P.quads);
   e = cudaGetLastError();
   return e == cudaSuccess ? SVG_OK : record_cuda_error("launch tile-map kernels", e);
 }

@@ -48,13 +48,15 @@ class svg_tile(ctypes.Structure):
 
 class svg_tilemap_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in ("total_bytes", "cls", "cnt", "row_ptr", "cols", "pair_ptr",
-                                               "pair_ent", "pair_cnt", "pair_order")] + \
-               [(n, ctypes.c_int32) for n in ("nq", "nk", "npairs", "reserved")]
+                                               "pair_ent", "pair_cnt", "pair_order", "quad_ptr", "quad_ent",
+                                               "quad_cnt", "quad_order")] + \
+               [(n, ctypes.c_int32) for n in ("nq", "nk", "npairs", "nquads")]
 
 
 class svg_tilemap_summary_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in ("retained_exact", "retained_map", "n_full", "n_boundary",
-                                               "n_empty", "visited_area", "pair_entries", "pair_half_tiles")]
+                                               "n_empty", "visited_area", "pair_entries", "pair_half_tiles",
+                                               "quad_entries", "quad_phase_tiles")]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -242,5 +244,9 @@ def tilemap_arrays(ws: torch.Tensor, geom: svg_geom, tile: svg_tile) -> dict:
         "pair_ent": u32(L.pair_ent, np_ * nk),
         "pair_cnt": u32(L.pair_cnt, 2 * np_).view(np_, 2),
         "pair_order": u32(L.pair_order, np_),
-        "nq": nq, "nk": nk, "npairs": np_,
+        "quad_ptr": u32(L.quad_ptr, L.nquads + 1),
+        "quad_ent": u32(L.quad_ent, L.nquads * nk),
+        "quad_cnt": u32(L.quad_cnt, 2 * L.nquads).view(L.nquads, 2),
+        "quad_order": u32(L.quad_order, L.nquads),
+        "nq": nq, "nk": nk, "npairs": np_, "nquads": L.nquads,
     }

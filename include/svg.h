@@ -86,7 +86,11 @@ typedef struct {
     uint64_t pair_ent;    /* uint32 [...]     kt | flagA << 28 | flagB << 30                  */
     uint64_t pair_cnt;    /* uint32 [2*np]    active entries of half 0 / half 1 of each pair  */
     uint64_t pair_order;  /* uint32 [np]      pairs by descending work, ties by index         */
-    int32_t nq, nk, npairs, reserved;
+    uint64_t quad_ptr;    /* uint32 [nquad+1] offsets of the 512-row (two-SM) execution lists  */
+    uint64_t quad_ent;    /* uint32 [...]     kt | flag(rank r, half h) << (24 + 4r + 2h)      */
+    uint64_t quad_cnt;    /* uint32 [2*nquad] entries where MMA phase 0 / phase 1 is active     */
+    uint64_t quad_order;  /* uint32 [nquad]   quads by descending work, ties by index           */
+    int32_t nq, nk, npairs, nquads;
 } svg_tilemap_layout;
 
 /* Totals of one built tile map (svg_tilemap_summary). */
@@ -97,6 +101,8 @@ typedef struct {
     uint64_t visited_area;    /* in-range pairs inside non-empty tiles                     */
     uint64_t pair_entries;    /* entries of all 256-row execution lists                    */
     uint64_t pair_half_tiles; /* active (entry, half) combinations: MMA work units          */
+    uint64_t quad_entries;    /* entries of all 512-row execution lists                    */
+    uint64_t quad_phase_tiles;/* active (entry, phase) combinations of the 512-row lists    */
 } svg_tilemap_summary_t;
 
 /*
@@ -112,9 +118,10 @@ int svg_tilemap_get_layout(svg_geom geom, svg_tile tile, svg_tilemap_layout *out
  * Classifies every (query tile, key tile) pair of one route class as full / boundary /
  * empty (rounded variant: full / empty), counts retained pairs per tile exactly, and
  * builds: the per-q-tile CSR list of visited tiles; the execution lists used by
- * svg_attention_fwd (one per 256-query-row pair of 128-row halves, with per-half flags
- * 0 skip, 1 full, 2 masked, 3 full but key range past the sequence end); and the pair
- * order by descending work used by its persistent scheduler. Integer work only.
+ * svg_attention_fwd, one per group of 128-row query blocks -- pairs (256 rows, one SM) and
+ * quads (512 rows, two SMs) -- with a flag per block: 0 skip, 1 full, 2 masked, 3 full but
+ * key range past the sequence end; and the group orders by descending work used by the
+ * persistent scheduler. Integer work only.
  *   d_ws: device buffer of at least svg_tilemap_bytes(geom, tile) bytes, 256-B aligned;
  *         written entirely by this call (also records the parameters it was built for).
  * Errors: SVG_ERR_ARG (bad geometry/mask/route), SVG_ERR_UNSUPPORTED (tile shape),

@@ -30,19 +30,21 @@ def u32(t):
     return t.cpu().numpy().view(np.uint32)
 
 
-def expected_pair_entries(cls, N, bq, bk):
-    """Execution lists derived from the class map (flags: 0 skip, 1 full, 2 masked, 3 full but
-    ragged key tile). A 128-row half combines the classes of the q-tiles it overlaps."""
+def expected_group_entries(cls, N, bq, bk, G):
+    """Execution lists derived from the class map for groups of G 128-row blocks (G = 2: pairs,
+    G = 4: quads). Block flag: 0 skip, 1 full, 2 masked, 3 full but ragged key tile; block i of a
+    group sits at bit 32 - 2G + 2i; per group, the entries in which MMA phase i % 2 is active."""
     nq, nk = cls.shape
-    npairs = -(-N // 256)
+    rows = 128 * G
+    ngroups = -(-N // rows)
     ragged = np.zeros(nk, dtype=bool)
     if N % bk:
         ragged[-1] = True
     ents, cnts = [], []
-    for p in range(npairs):
+    for p in range(ngroups):
         flags = []
-        for h in range(2):
-            r0 = 256 * p + 128 * h
+        for i in range(G):
+            r0 = rows * p + 128 * i
             if r0 >= N:
                 flags.append(np.zeros(nk, dtype=np.uint32))
                 continue
@@ -50,13 +52,34 @@ def expected_pair_entries(cls, N, bq, bk):
             cs = cls[r0 // bq: (r1 - 1) // bq + 1]
             anyk = (cs != 0).any(axis=0)
             allf = (cs == 1).all(axis=0)
-            f = np.where(~anyk, 0, np.where(allf, np.where(ragged, 3, 1), 2)).astype(np.uint32)
-            flags.append(f)
-        act = (flags[0] | flags[1]) != 0
-        kts = np.nonzero(act)[0].astype(np.uint32)
-        ents.append(kts | (flags[0][act] << 28) | (flags[1][act] << 30))
-        cnts.append((int((flags[0] != 0).sum()), int((flags[1] != 0).sum())))
+            flags.append(np.where(~anyk, 0, np.where(allf, np.where(ragged, 3, 1), 2)).astype(np.uint32))
+        phase = [np.zeros(nk, dtype=bool), np.zeros(nk, dtype=bool)]
+        for i in range(G):
+            phase[i % 2] |= flags[i] != 0
+        act = phase[0] | phase[1]
+        e = np.nonzero(act)[0].astype(np.uint32)
+        for i in range(G):
+            e = e | (flags[i][act] << np.uint32(32 - 2 * G + 2 * i))
+        ents.append(e)
+        cnts.append((int(phase[0].sum()), int(phase[1].sum())))
     return ents, cnts
+
+
+def check_group_lists(A, summ, cls, N, bq, bk, G):
+    key = "pair" if G == 2 else "quad"
+    ents, cnts = expected_group_entries(cls, N, bq, bk, G)
+    ptr = u32(A[key + "_ptr"]).astype(np.int64)
+    ent = u32(A[key + "_ent"])
+    cnt = u32(A[key + "_cnt"]).reshape(-1, 2)
+    for p in range(len(ents)):
+        assert np.array_equal(ent[ptr[p]: ptr[p + 1]], ents[p]), (key, p)
+        assert tuple(cnt[p]) == cnts[p], (key, p)
+    work = cnt.sum(axis=1).astype(np.int64)
+    order = u32(A[key + "_order"]).astype(np.int64)
+    assert np.array_equal(order, np.lexsort((np.arange(len(work)), -work)))
+    tot_e = summ.pair_entries if G == 2 else summ.quad_entries
+    tot_w = summ.pair_half_tiles if G == 2 else summ.quad_phase_tiles
+    assert tot_e == sum(len(e) for e in ents) and tot_w == int(work.sum())
 
 
 def check_tilemap(S, w, route, variant, bq, bk, qts=None):
@@ -98,20 +121,9 @@ def check_tilemap(S, w, route, variant, bq, bk, qts=None):
         kts = np.nonzero(cls[qt])[0]
         assert np.array_equal(seg & 0x3FFFFFFF, kts)
         assert np.array_equal(seg >> 30, cls[qt, kts])
-    # execution lists and scheduler order (derived from the map, which matched the oracle)
-    ents, cnts = expected_pair_entries(cls, N, bq, bk)
-    pptr = u32(A["pair_ptr"]).astype(np.int64)
-    pent = u32(A["pair_ent"])
-    pcnt = u32(A["pair_cnt"]).reshape(-1, 2)
-    for p in range(A["npairs"]):
-        assert np.array_equal(pent[pptr[p]: pptr[p + 1]], ents[p]), p
-        assert tuple(pcnt[p]) == cnts[p]
-    work = pcnt.sum(axis=1).astype(np.int64)
-    order = u32(A["pair_order"]).astype(np.int64)
-    assert np.array_equal(np.sort(order), np.arange(A["npairs"]))
-    assert np.array_equal(order, np.lexsort((np.arange(len(work)), -work)))
-    assert summ.pair_entries == sum(len(e) for e in ents)
-    assert summ.pair_half_tiles == int(work.sum())
+    # execution lists and scheduler orders (derived from the map, which matched the oracle)
+    check_group_lists(A, summ, cls, N, bq, bk, 2)
+    check_group_lists(A, summ, cls, N, bq, bk, 4)
     return summ
 
 
