@@ -392,6 +392,13 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
         out[f"{name}_boundary_frac_of_visited"] = bnd / max(vis, 1)
         out[f"{name}_visited_frac_of_all"] = vis / max(tot_tiles, 1)
         out[f"{name}_retained_frac"] = kept / (w.heads * w.tokens ** 2)
+    # head routing from 64 sampled query rows per head (original order, dense + both sparse masks)
+    rows = torch.as_tensor(syn.sample_rows(w.replace(sample_rows=64), 0)[:64].numpy(), dtype=torch.int32,
+                           device=dev)
+    rt = torch.empty(w.heads, dtype=torch.uint8, device=dev)
+    work = torch.empty(S.svg_route_work_bytes(w.heads, rows.numel()), dtype=torch.uint8, device=dev)
+    out["route_ms"] = time_events(lambda: S.svg_route_heads(q, k, v, g, m, rows, rt, work=work), 5, stream)
+    out["route_rows_per_head"] = int(rows.numel())
     st = S.svg_read_status(scratch)
     out["status"] = st
     return out

@@ -112,3 +112,29 @@ def sample_rows(w: Workload, head: int, seed: int = 1234) -> torch.Tensor:
     fixed = torch.tensor([0, 1, n // 2, n - 2, n - 1], dtype=torch.int64)
     tail = torch.arange(max(0, n - 96), n, dtype=torch.int64)
     return torch.unique(torch.cat([r, fixed, tail]))
+
+
+def make_routed_qkv(w: Workload, kinds, strength: float = 1.5, seed_offset: int = 0, dtype=torch.bfloat16):
+    """Q/K/V with planted head structure, original order, for routing checks.
+
+    kinds[h] = ROUTE_SPATIAL: every frame has its own random direction, added (times `strength`)
+    to the queries and keys of that frame, so a query's largest scores are within its frame.
+    kinds[h] = ROUTE_TEMPORAL: every patch position has its own direction instead, so a query's
+    largest scores are at its patch across frames. V is plain N(0, 1)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(100 + seed_offset)
+    T, S, N, d = w.frames, w.frame_size, w.tokens, w.d
+    q = torch.randn((w.heads, N, d), generator=g)
+    k = torch.randn((w.heads, N, d), generator=g)
+    v = torch.randn((w.heads, N, d), generator=g)
+    tok = torch.arange(N)
+    for h, kind in enumerate(kinds):
+        if kind == ROUTE_SPATIAL:
+            dirs = torch.randn((T, d), generator=g)
+            idx = tok // S
+        else:
+            dirs = torch.randn((S, d), generator=g)
+            idx = tok % S
+        q[h] += strength * dirs[idx]
+        k[h] += strength * dirs[idx]
+    return q.to(dtype), k.to(dtype), v.to(dtype)

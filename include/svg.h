@@ -209,6 +209,27 @@ int svg_attention_fwd_noalloc(const void *q, const void *k, const void *v, void 
                               const void *d_ws_temporal, svg_geom geom, svg_mask mask,
                               svg_tile tile, int32_t mode, int32_t *d_status, void *stream);
 
+/*
+ * Head routing by sampling: Sparse VideoGen profiles heads at inference time and routes each to
+ * the spatial or the temporal mask based on sampled rows ("Sparse Attention Patterns"; summary of
+ * the case study). For every head, the query rows listed in d_rows (ORIGINAL token indices,
+ * frame-major) attend to all keys under the dense mask, the spatial mask and the temporal mask of
+ * `mask` (exact variant, original token order; layout and variant are ignored), in fp32. With
+ * E_m = sum over the rows of |O_m - O_dense|^2 and E_d = sum of |O_dense|^2:
+ *   d_route[h] = E_spatial <= E_temporal ? SVG_ROUTE_SPATIAL : SVG_ROUTE_TEMPORAL
+ *   d_err[2h], d_err[2h+1] = E_spatial / E_d, E_temporal / E_d   (d_err nullable)
+ *   q, k, v:  [heads, tokens, d] bf16 in ORIGINAL order (before any permutation).
+ *   d_rows:   device int32 [n_rows]; entries outside [0, tokens) are ignored.
+ *   d_work:   device buffer of svg_route_work_bytes(heads, n_rows) bytes (per-row errors).
+ *   d_route:  device uint8 [heads].
+ * The sums over rows run in a fixed order, so the decision is deterministic.
+ */
+size_t svg_route_work_bytes(int32_t heads, int32_t n_rows);
+int svg_route_heads(const void *q, const void *k, const void *v, int32_t heads, int64_t tokens,
+                    int32_t d, float scale, svg_geom geom, svg_mask mask, const int32_t *d_rows,
+                    int32_t n_rows, void *d_work, size_t work_bytes, uint8_t *d_route,
+                    float *d_err, void *stream);
+
 /* Reads the device status word of a scratch buffer (or d_status). Synchronises `stream`. */
 int svg_read_status(const void *d_scratch_or_status, int32_t *h_status, void *stream);
 

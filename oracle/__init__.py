@@ -12,6 +12,8 @@ Parity status of each routine (what pins it, in tests/test_oracle_pins.py):
                                         V=1 => O=1 (rows sum to 1); LSE(Q=0) = ln(#kept);
                                         numpy brute force with an explicit N x N mask
   or_perm_table                 pinned: bijection, closed-form positions of corner tokens
+  or_route_errors               pinned: masks equal to dense give zero error; constant V gives a
+                                        tie; planted spatial / temporal structure is recovered
 """
 from __future__ import annotations
 
@@ -65,6 +67,8 @@ def lib():
                                         i64, ctypes.c_int, ctypes.c_void_p, i64, i64, i64p, i64,
                                         ctypes.c_void_p, ctypes.c_void_p]
         L.or_num_threads.restype = ctypes.c_int
+        L.or_route_errors.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, i64, i64, ctypes.c_double,
+                                      i64, i64, i64, i64, i64, i64p, i64, ctypes.c_void_p]
         _lib = L
     return _lib
 
@@ -162,3 +166,28 @@ def attention_rows(q, k, v, rows, *, route, layout, T, S, frame_window, band, F0
                             rc.ctypes.data if rc is not None else None, bq, bk,
                             _p(rows, ctypes.c_int64), len(rows), out.ctypes.data, lse.ctypes.data)
     return out, lse
+
+
+def _bits(x):
+    import torch
+    if isinstance(x, torch.Tensor):
+        return np.ascontiguousarray(x.contiguous().view(torch.int16).numpy().view(np.uint16))
+    return np.ascontiguousarray(x, dtype=np.uint16)
+
+
+def route_errors(q, k, v, rows, *, T, S, frame_window, band, F0, scale=None):
+    """(E_spatial, E_temporal, E_dense) of one head over the sampled original rows (fp64)."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    N, d = qb.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.empty(3, dtype=np.float64)
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(d)
+    lib().or_route_errors(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, N, d, float(scale), T, S, frame_window,
+                          band, F0, _p(rows, ctypes.c_int64), len(rows), out.ctypes.data)
+    return float(out[0]), float(out[1]), float(out[2])
+
+
+def route(q, k, v, rows, **kw) -> int:
+    es, et, _ = route_errors(q, k, v, rows, **kw)
+    return ROUTE_SPATIAL if es <= et else ROUTE_TEMPORAL

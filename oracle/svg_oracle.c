@@ -223,6 +223,35 @@ void or_attention_rows(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
     free(pi); free(kd); free(vd);
 }
 
+/*
+ * Head routing by sampled rows (Sparse VideoGen's inference-time profiling, read as: attend the
+ * sampled rows under the dense, spatial and temporal masks and compare with dense):
+ *   out[0] = sum_rows |O_spatial - O_dense|^2, out[1] = sum_rows |O_temporal - O_dense|^2,
+ *   out[2] = sum_rows |O_dense|^2  (fp64; exact masks on original identities).
+ * The route is spatial iff out[0] <= out[1].
+ */
+void or_route_errors(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int64_t N, int64_t d, double scale,
+                     int64_t T, int64_t S, int64_t k, int64_t b, int64_t F0, const int64_t *rows, int64_t n_rows,
+                     double *out) {
+    double *od = (double *)malloc(sizeof(double) * (size_t)(n_rows * d));
+    double *os = (double *)malloc(sizeof(double) * (size_t)(n_rows * d));
+    double *ot = (double *)malloc(sizeof(double) * (size_t)(n_rows * d));
+    double *lse = (double *)malloc(sizeof(double) * (size_t)n_rows);
+    or_attention_rows(q, kk, v, N, d, scale, OR_ROUTE_SPATIAL, 0, T, S, k, b, F0, 2, NULL, 1, 1, rows, n_rows, od, lse);
+    or_attention_rows(q, kk, v, N, d, scale, OR_ROUTE_SPATIAL, 0, T, S, k, b, F0, 0, NULL, 1, 1, rows, n_rows, os, lse);
+    or_attention_rows(q, kk, v, N, d, scale, OR_ROUTE_TEMPORAL, 0, T, S, k, b, F0, 0, NULL, 1, 1, rows, n_rows, ot, lse);
+    double es = 0.0, et = 0.0, ed = 0.0;
+    for (int64_t x = 0; x < n_rows * d; ++x) {
+        es += (os[x] - od[x]) * (os[x] - od[x]);
+        et += (ot[x] - od[x]) * (ot[x] - od[x]);
+        ed += od[x] * od[x];
+    }
+    out[0] = es;
+    out[1] = et;
+    out[2] = ed;
+    free(od); free(os); free(ot); free(lse);
+}
+
 /* Threads the OpenMP runtime will use (reported next to oracle timings). */
 int or_num_threads(void) {
 #ifdef _OPENMP

@@ -296,3 +296,67 @@ def test_attention_pages_mixed_naive(S):
 
 def test_attention_1440p(S):
     _pages(syn.P1440, rows=256)
+
+
+# ----------------------------------------------------------------------------- head routing
+def _route_case(S, w, q, k, v, rows):
+    g, m, _ = gp.geom_mask_tile(w)
+    dev = "cuda"
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    rd = torch.as_tensor(np.asarray(rows), dtype=torch.int32, device=dev)
+    route = torch.full((w.heads,), 255, dtype=torch.uint8, device=dev)
+    err = torch.full((w.heads, 2), -1.0, dtype=torch.float32, device=dev)
+    S.svg_route_heads(qd, kd, vd, g, m, rd, route, err)
+    torch.cuda.synchronize()
+    valid = [r for r in np.asarray(rows).tolist() if 0 <= r < w.tokens]
+    want_err, want_route = [], []
+    for h in range(w.heads):
+        es, et, ed = oracle.route_errors(q[h], k[h], v[h], valid, T=w.frames, S=w.frame_size,
+                                         frame_window=w.frame_window, band=w.spatial_band, F0=w.sink_frames)
+        want_err.append((es / ed, et / ed))
+        want_route.append(0 if es <= et else 1)
+    return route.cpu().numpy(), err.cpu().numpy().astype(np.float64), np.array(want_route), np.array(want_err)
+
+
+def _check_routes(got_r, got_e, want_r, want_e):
+    # fp32 accumulation against fp64: relative errors within 1e-3 of their own size
+    assert np.allclose(got_e, want_e, rtol=2e-3, atol=1e-6), (got_e, want_e)
+    for h in range(len(want_r)):
+        es, et = want_e[h]
+        if abs(es - et) > 1e-2 * max(es, et):
+            assert got_r[h] == want_r[h], (h, got_r, want_r)
+        else:  # a near tie may go either way; the decision must match the device's own errors
+            assert got_r[h] == (0 if got_e[h][0] <= got_e[h][1] else 1)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_route_planted_structure(S, d):
+    w = syn.Workload("route_medium", frames=6, grid_h=8, grid_w=12, routes=(0, 1, 1, 0, 1, 0), d=d,
+                     frame_window=1, spatial_band=2)
+    kinds = list(w.routes)
+    q, k, v = syn.make_routed_qkv(w, kinds, seed_offset=d)
+    rows = np.arange(0, w.tokens, 3)  # 192 rows: a ragged last block of sampled rows
+    got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
+    _check_routes(got_r, got_e, want_r, want_e)
+    assert list(got_r) == kinds == list(want_r)
+
+
+def test_route_random_heads_and_rows_outside(S):
+    """Unstructured heads (decisions follow the oracle's errors) and sampled rows that fall outside
+    the sequence, which contribute nothing."""
+    w = MEDIUM
+    q, k, v = syn.make_qkv(w, seed_offset=11)
+    rows = np.concatenate([np.arange(0, w.tokens, 13), [-1, w.tokens, w.tokens + 5]])
+    got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
+    _check_routes(got_r, got_e, want_r, want_e)
+
+
+def test_route_pages_shape(S):
+    """Routing at 75,600 tokens with 64 sampled rows per head, planted spatial and temporal heads."""
+    w = syn.MIXED_75K.replace(routes=(0, 1, 0, 1))
+    kinds = list(w.routes)
+    q, k, v = syn.make_routed_qkv(w, kinds, strength=1.0, seed_offset=3)
+    rows = syn.sample_rows(w.replace(sample_rows=64), 0).numpy()
+    got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
+    _check_routes(got_r, got_e, want_r, want_e)
+    assert list(got_r) == kinds

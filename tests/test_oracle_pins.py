@@ -381,3 +381,42 @@ def test_rounded_mask_attention_matches_explicit_tile_mask():
         ref, _ = numpy_masked_attention(f64(q)[has], f64(k), f64(v), mask[has], 1 / math.sqrt(d))
         np.testing.assert_allclose(out[has], ref, rtol=1e-10, atol=1e-12)
         assert np.all(out[~has] == 0)
+
+
+# ----------------------------------------------------------------------------- head routing
+def test_route_masks_equal_to_dense_have_zero_error():
+    """A spatial window covering every frame keeps every pair, so E_spatial = 0 exactly; a
+    patch band covering every patch does the same for E_temporal."""
+    w = syn.Workload("r", frames=4, grid_h=4, grid_w=6, routes=(0,), d=32, frame_window=1, spatial_band=2)
+    q, k, v = syn.make_qkv(w, seed_offset=4)
+    rows = np.arange(0, w.tokens, 5)
+    es, et, ed = oracle.route_errors(q[0], k[0], v[0], rows, T=4, S=24, frame_window=4, band=2, F0=1)
+    assert es == 0.0 and et > 0.0 and ed > 0.0
+    es, et, ed = oracle.route_errors(q[0], k[0], v[0], rows, T=4, S=24, frame_window=1, band=24, F0=1)
+    assert et == 0.0 and es > 0.0
+    assert oracle.route(q[0], k[0], v[0], rows, T=4, S=24, frame_window=1, band=24, F0=1) == syn.ROUTE_TEMPORAL
+
+
+def test_route_constant_values_and_ties():
+    w = syn.Workload("r", frames=3, grid_h=4, grid_w=4, routes=(0,), d=16, frame_window=0, spatial_band=1)
+    q, k, _ = syn.make_qkv(w, seed_offset=6)
+    v = bf16(torch.full((w.tokens, w.d), 0.75))
+    es, et, ed = oracle.route_errors(q[0], k[0], v, np.arange(w.tokens), T=3, S=16, frame_window=0, band=1, F0=1)
+    # every mask averages the same constant: both errors are rounding noise only
+    assert es < 1e-20 and et < 1e-20 and abs(ed - w.tokens * w.d * 0.5625) < 1e-9
+    # both masks keep every pair: the errors are exactly equal (zero) and the tie goes spatial
+    es, et, _ = oracle.route_errors(q[0], k[0], v, np.arange(w.tokens), T=3, S=16, frame_window=3, band=16, F0=1)
+    assert es == et == 0.0
+    assert oracle.route(q[0], k[0], v, np.arange(w.tokens), T=3, S=16, frame_window=3, band=16, F0=1) == 0
+
+
+def test_route_recovers_planted_structure():
+    w = syn.Workload("r", frames=6, grid_h=8, grid_w=8, routes=(0, 1, 1, 0), d=64, frame_window=1, spatial_band=2)
+    kinds = [0, 1, 1, 0]
+    q, k, v = syn.make_routed_qkv(w, kinds)
+    rows = np.arange(0, w.tokens, 7)
+    for h, kind in enumerate(kinds):
+        kw = dict(T=w.frames, S=w.frame_size, frame_window=1, band=2, F0=1)
+        es, et, _ = oracle.route_errors(q[h], k[h], v[h], rows, **kw)
+        assert oracle.route(q[h], k[h], v[h], rows, **kw) == kind, (h, es, et)
+        assert (es < 0.5 * et) if kind == 0 else (et < 0.5 * es)
