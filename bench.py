@@ -297,7 +297,7 @@ def main():
     peak = float(P["bf16_tflops"])
     achieved = vis_flop / (statistics.mean(per_step) * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": captured_traffic(w, args),
                 "kernel": "attn_kernel<128,128> (split)", "flop_definition": "4*d*(in-range area of visited tiles)",
                 "peak_kind": f"{peak_kind} bf16 burst"}
 
@@ -343,6 +343,32 @@ def main():
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+# DRAM bytes (read + write) of one attention launch from an ncu capture of the 2-head slice of
+# spatial_75600 (128 x 128 tiles, split mode), scaled to the launch's heads: traffic grows with the
+# heads processed. Valid only for the kernel sources that were captured (their SHA-256 prefix);
+# after any change to them the field is null until the capture is repeated.
+CAPTURED_TRAFFIC = {"sources_sha256": "f9bae6f0246475ef", "bytes_per_head": 146.244e6 / 2,
+                    "workload": "spatial_75600", "bq": 128, "bk": 128, "mode": "split"}
+
+
+def kernel_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_spatio_flash_b200", "csrc")
+    for name in ("svg_attention.cu", "svg_common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(w, args):
+    c = CAPTURED_TRAFFIC
+    if (kernel_sources_sha() != c["sources_sha256"] or w.name != c["workload"] or args.bq != c["bq"]
+            or args.bk != c["bk"] or args.mode != c["mode"]):
+        return None
+    return c["bytes_per_head"] * w.heads
 
 
 def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws, summ, P, stream, dev):
@@ -396,7 +422,7 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
     rows = torch.as_tensor(syn.sample_rows(w.replace(sample_rows=64), 0)[:64].numpy(), dtype=torch.int32,
                            device=dev)
     rt = torch.empty(w.heads, dtype=torch.uint8, device=dev)
-    work = torch.empty(S.svg_route_work_bytes(w.heads, rows.numel()), dtype=torch.uint8, device=dev)
+    work = torch.empty(S.svg_route_work_bytes(w.heads, w.tokens, w.d, rows.numel()), dtype=torch.uint8, device=dev)
     out["route_ms"] = time_events(lambda: S.svg_route_heads(q, k, v, g, m, rows, rt, work=work), 5, stream)
     out["route_rows_per_head"] = int(rows.numel())
     st = S.svg_read_status(scratch)

@@ -17,8 +17,9 @@ int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const
                    svg_mask mask, int inverse, int num_sms, cudaStream_t st);
 int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st);
 int launch_attention_pair(const AttnParams& P, int bk, int max_clusters, cudaStream_t st);
+size_t route_work_bytes(int heads, int64_t N, int d, int n_rows);
 int launch_route(const void* q, const void* k, const void* v, int heads, int N, int d, float scale, svg_geom geom,
-                 svg_mask mask, const int32_t* rows, int n_rows, float* work, uint8_t* route, float* err,
+                 svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
                  cudaStream_t st);
 }  // namespace svg
 
@@ -400,9 +401,9 @@ int svg_attention_fwd_noalloc(const void* q, const void* k, const void* v, void*
                        static_cast<cudaStream_t>(stream));
 }
 
-size_t svg_route_work_bytes(int32_t heads, int32_t n_rows) {
-  if (heads < 1 || n_rows < 1) return 0;
-  return (size_t)heads * (size_t)n_rows * 3 * sizeof(float);
+size_t svg_route_work_bytes(int32_t heads, int64_t tokens, int32_t d, int32_t n_rows) {
+  if (heads < 1 || n_rows < 1 || tokens < 1 || tokens > INT32_MAX || (d != 64 && d != 128)) return 0;
+  return route_work_bytes(heads, tokens, d, n_rows);
 }
 
 int svg_route_heads(const void* q, const void* k, const void* v, int32_t heads, int64_t tokens, int32_t d, float scale,
@@ -415,12 +416,12 @@ int svg_route_heads(const void* q, const void* k, const void* v, int32_t heads, 
   if (heads < 1 || heads > 65535 || n_rows < 1 || !geom_ok(geom) || !mask_ok(geom, mask)) return SVG_ERR_ARG;
   if ((int64_t)geom.frames * geom.grid_h * geom.grid_w != tokens) return SVG_ERR_ARG;
   if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
-  if (work_bytes < svg_route_work_bytes(heads, n_rows)) return SVG_ERR_WORKSPACE;
+  if (work_bytes < svg_route_work_bytes(heads, tokens, d, n_rows)) return SVG_ERR_WORKSPACE;
   int rc = device_info(nullptr);
   if (rc) return rc;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
-  return launch_route(q, k, v, heads, (int)tokens, d, sc, geom, mask, d_rows, n_rows, static_cast<float*>(d_work),
-                      d_route, d_err, static_cast<cudaStream_t>(stream));
+  return launch_route(q, k, v, heads, (int)tokens, d, sc, geom, mask, d_rows, n_rows, d_work, d_route, d_err,
+                      static_cast<cudaStream_t>(stream));
 }
 
 int svg_read_status(const void* d_scratch_or_status, int32_t* h_status, void* stream) {

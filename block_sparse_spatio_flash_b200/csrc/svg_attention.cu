@@ -176,6 +176,98 @@ __device__ ItemInfo decode_item(const AttnParams& P, uint32_t idx) {
 }
 
 // ---------------------------------------------------------------------------------------
+// Softmax steps of one score row (one thread per query row, BK scores in registers).
+
+// The row's BK fp32 scores from TMEM.
+template <int BK>
+__device__ __forceinline__ void load_scores(uint32_t tS, uint32_t* r) {
+#pragma unroll
+  for (int q = 0; q < BK / 32; ++q) tmem_ld32(tS + q * 32, r + q * 32);
+  tmem_ld_wait();
+#pragma unroll
+  for (int q = 0; q < BK / 32; ++q) tmem_ld_fence32(r + q * 32);
+}
+
+// Sets to -inf the scores the mask drops: boundary tiles element by element (kept keys of the
+// row are [0, se) U [lo, hi), or the periodic sink of the fully space-major order), the ragged
+// key tail, every visited tile in naive mode, and rows without a kept tile under rounded masks.
+template <int BK>
+__device__ __forceinline__ void mask_scores(const AttnParams& P, int cls, uint32_t f, int c0, int prow, uint32_t ent,
+                                            int lo, int hi, int se, bool per, uint32_t* r) {
+  float* s = reinterpret_cast<float*>(r);
+  const bool elem = (f == kFlagMasked) || (P.naive && !P.dense);
+  if (!(elem || f == kFlagBounds)) return;
+  const int nn = P.N - c0;
+  if (!elem) {
+#pragma unroll
+    for (int j = 0; j < BK; ++j)
+      if (j >= nn) s[j] = -INFINITY;
+  } else if (P.variant == SVG_MASK_ROUNDED) {
+    const uint8_t* rcls = P.cls[cls] + (size_t)(prow / P.bq) * P.nk;
+    const bool rowkept = __ldg(rcls + ent_kt(ent)) == 1;
+#pragma unroll
+    for (int j = 0; j < BK; ++j)
+      if (!(rowkept && j < nn)) s[j] = -INFINITY;
+  } else {
+    const int a = lo - c0;
+    const uint32_t w = (uint32_t)(hi - lo);
+    const int sk = se - c0;
+    if (!per) {
+#pragma unroll
+      for (int j = 0; j < BK; ++j) {
+        const bool keep = (j < nn) && ((j < sk) || ((uint32_t)(j - a) < w));
+        if (!keep) s[j] = -INFINITY;
+      }
+    } else {
+      const MaskGeom& g = P.g[cls];
+      int rr = c0 % g.T;
+#pragma unroll
+      for (int j = 0; j < BK; ++j) {
+        const bool keep = (j < nn) && ((rr < g.F0) || ((uint32_t)(j - a) < w));
+        if (!keep) s[j] = -INFINITY;
+        rr = (rr + 1 == g.T) ? 0 : rr + 1;
+      }
+    }
+  }
+}
+
+// Row maximum first, then the rescale decision: the warp rescales (returns true) when any row's
+// maximum grew by more than 2^kRescaleThreshold or had none yet; l is corrected here, O by the
+// caller after P is stored.
+template <int BK>
+__device__ __forceinline__ bool max_first(const uint32_t* r, float sl2, float& m, float& l, float& alpha) {
+  const float* s = reinterpret_cast<const float*>(r);
+  float mx4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mx4[i] = s[i];
+#pragma unroll
+  for (int j = 4; j < BK; j += 4)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(mx4[i], s[j + i]);
+  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  const float m_new = fmaxf(m, mx);
+  const bool need = (m_new > m) && (m == -INFINITY || (m_new - m) * sl2 > kRescaleThreshold);
+  const bool rescale = __any_sync(0xffffffffu, need);
+  if (rescale) {
+    alpha = (m_new == -INFINITY) ? 1.f : ex2f((m - m_new) * sl2);
+    l *= alpha;
+    m = m_new;
+  }
+  return rescale;
+}
+
+// P = 2^(S * sl2 - m * sl2) packed to bf16 into r[0, BK/2), fp32 partial row sums in acc.
+template <int BK>
+__device__ __forceinline__ void exp_tile(uint32_t* r, float sl2, float m, float2 (&acc)[2]) {
+  const float base = (m == -INFINITY) ? 0.f : m * sl2;
+  const float2 sc = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+  acc[0] = make_float2(0.f, 0.f);
+  acc[1] = make_float2(0.f, 0.f);
+  exp_pack_64<0>(r, sc, nb, acc);
+  if (BK == 128) exp_pack_64<64 % BK>(r, sc, nb, acc);
+}
+
+// ---------------------------------------------------------------------------------------
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
   using C = Cfg<D, BK>;
@@ -453,80 +545,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         ++s_cnt;
         tc_fence_after();
         uint32_t r[BK];
-#pragma unroll
-        for (int q = 0; q < BK / 32; ++q) tmem_ld32(tS + q * 32, r + q * 32);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < BK / 32; ++q) tmem_ld_fence32(r + q * 32);
-        float* s = reinterpret_cast<float*>(r);
-        // ---- masking (boundary tiles, ragged key tail, naive mode)
-        const bool elem = (f == kFlagMasked) || (P.naive && !P.dense);
-        if (elem || f == kFlagBounds) {
-          const int nn = P.N - c0;
-          if (!elem) {
-#pragma unroll
-            for (int j = 0; j < BK; ++j)
-              if (j >= nn) s[j] = -INFINITY;
-          } else if (P.variant == SVG_MASK_ROUNDED) {
-            const uint8_t* rcls = P.cls[inf.cls] + (size_t)(prow / P.bq) * P.nk;
-            const bool rowkept = __ldg(rcls + ent_kt(ent)) == 1;
-#pragma unroll
-            for (int j = 0; j < BK; ++j)
-              if (!(rowkept && j < nn)) s[j] = -INFINITY;
-          } else {
-            const int a = lo - c0;
-            const uint32_t w = (uint32_t)(hi - lo);
-            const int sk = se - c0;
-            if (!per) {
-#pragma unroll
-              for (int j = 0; j < BK; ++j) {
-                const bool keep = (j < nn) && ((j < sk) || ((uint32_t)(j - a) < w));
-                if (!keep) s[j] = -INFINITY;
-              }
-            } else {
-              const MaskGeom& g = P.g[inf.cls];
-              int rr = c0 % g.T;
-#pragma unroll
-              for (int j = 0; j < BK; ++j) {
-                const bool keep = (j < nn) && ((rr < g.F0) || ((uint32_t)(j - a) < w));
-                if (!keep) s[j] = -INFINITY;
-                rr = (rr + 1 == g.T) ? 0 : rr + 1;
-              }
-            }
-          }
-        }
-        // ---- online softmax: row max and row sum as independent chains
-        float mx4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) mx4[i] = s[i];
-#pragma unroll
-        for (int j = 4; j < BK; j += 4)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(mx4[i], s[j + i]);
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        const float m_new = fmaxf(m, mx);
-        const bool need = (m_new > m) && (m == -INFINITY || (m_new - m) * sl2 > kRescaleThreshold);
-        // the O correction itself runs after P is stored, when the score row is dead
-        const bool rescale = __any_sync(0xffffffffu, need);
         float alpha = 1.f;
-        if (rescale) {
-          alpha = (m_new == -INFINITY) ? 1.f : ex2f((m - m_new) * sl2);
-          l *= alpha;
-          m = m_new;
-        }
-        const float base = (m == -INFINITY) ? 0.f : m * sl2;
-        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < BK; j += 2) {
-          const float x0 = fmaf(s[j], sl2, -base);
-          const float x1 = fmaf(s[j + 1], sl2, -base);
-          const float p0 = ((kPolyMask >> (j & 7)) & 1u) ? exp2_poly(x0) : ex2f(x0);
-          const float p1 = ((kPolyMask >> ((j + 1) & 7)) & 1u) ? exp2_poly(x1) : ex2f(x1);
-          ls4[j & 3] += p0;
-          ls4[(j + 1) & 3] += p1;
-          r[j / 2] = pack_bf16(p0, p1);  // packed P overwrites the consumed front of the row
-        }
-        l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+        float2 acc[2];
+        load_scores<BK>(tS, r);
+        mask_scores<BK>(P, inf.cls, f, c0, prow, ent, lo, hi, se, per, r);
+        const bool rescale = max_first<BK>(r, sl2, m, l, alpha);
+        exp_tile<BK>(r, sl2, m, acc);
+        l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
 #pragma unroll
         for (int q = 0; q < BK / 64; ++q) tmem_st32(tP + q * 32, r + q * 32);
         if (rescale && !first) {  // O_h holds every earlier P V (S_h's commit covered them)
@@ -551,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       if (!__all_sync(0xffffffffu, wait_bar(c.o_done(h), od_cnt & 1u, abort_addr, status))) break;
       ++od_cnt;
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = (l > 0.f && m != -INFINITY) ? 1.f / l : 0.f;  // a row with no kept key gives 0
       __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + prow) * D;
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
@@ -576,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       mbar_arrive(c.o_free(h));
       if (in_range && P.lse)
         P.lse[(size_t)inf.head * P.N + row] =
-            l > 0.f ? (m * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            (l > 0.f && m != -INFINITY) ? (m * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 

@@ -540,20 +540,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           m = m_new;
         }
         const float base = (m == -INFINITY) ? 0.f : m * sl2;
-        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const float2 sc = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+          float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          exp_pack_64<0>(r, sc, nb, acc);
+          if (BK == 128) exp_pack_64<64 % BK>(r, sc, nb, acc);
 #pragma unroll
-        for (int j = 0; j < BK; j += 2) {
-          const float x0 = fmaf(s[j], sl2, -base);
-          const float x1 = fmaf(s[j + 1], sl2, -base);
-          const float p0 = ((kPolyMask >> (j & 7)) & 1u) ? exp2_poly(x0) : ex2f(x0);
-          const float p1 = ((kPolyMask >> ((j + 1) & 7)) & 1u) ? exp2_poly(x1) : ex2f(x1);
-          ls4[j & 3] += p0;
-          ls4[(j + 1) & 3] += p1;
-          r[j / 2] = pack_bf16(p0, p1);
+          for (int q = 0; q < BK / 64; ++q) tmem_st32(tP + q * 32, r + q * 32);
+          l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
         }
-        l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-#pragma unroll
-        for (int q = 0; q < BK / 64; ++q) tmem_st32(tP + q * 32, r + q * 32);
         if (rescale && !first) {
 #pragma unroll 1
           for (int q = 0; q < D / 32; ++q) {
@@ -575,7 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, wait_bar(c.o_done(c.base, h), od_cnt & 1u, ab))) break;
       ++od_cnt;
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = (l > 0.f && m != -INFINITY) ? 1.f / l : 0.f;  // a row with no kept key gives 0
       __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + prow) * D;
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
@@ -600,7 +595,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_arrive_cluster(c.o_free(c.lead, h));
       if (in_range && P.lse)
         P.lse[(size_t)inf.head * P.N + row] =
-            l > 0.f ? (m * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            (l > 0.f && m != -INFINITY) ? (m * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 

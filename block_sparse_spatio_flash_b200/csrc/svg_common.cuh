@@ -484,7 +484,9 @@ __device__ __forceinline__ float ex2f(float x) {
 // Cody-Waite style range reduction: n = round(x) (by the 1.5*2^23 rounding trick), f = x - n in
 // [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
 // error on [-1/2, 1/2] (fitted by linear programming, max rel. error 7.5e-5, far below the bf16
-// rounding of P); 2^n is added to the exponent field. Exact 0 for x < -125 (masked scores).
+// rounding of P); 2^n is added to the exponent field by one integer multiply-add. Inputs below
+// -125 (masked scores are -inf) give 2^-125 times the polynomial's value at 0, a normal number
+// too small to move any finite sum; a row whose every score is masked is zeroed by its caller.
 constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f, kExpC2 = 2.426111251e-01f,
                 kExpC3 = 5.517166853e-02f;
 __device__ __forceinline__ float exp2_poly(float x) {
@@ -493,19 +495,52 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const float n = r - 12582912.f;
   const float f = xc - n;
   const float p = fmaf(fmaf(fmaf(kExpC3, f, kExpC2), f, kExpC1), f, kExpC0);
-  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
-  return x < -125.f ? 0.f : y;
+  return __uint_as_float((__float_as_uint(r) << 23) + __float_as_uint(p));
 }
 
-// Columns (mod 8) whose exponential is computed by exp2_poly instead of ex2.approx.
+// Column pairs (mod 8) whose exponentials are computed by exp2_poly2 instead of ex2.approx.
 #ifndef SVG_POLY_MASK
 #define SVG_POLY_MASK 0x00u
 #endif
 constexpr uint32_t kPolyMask = SVG_POLY_MASK;
 
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low 16 bits)
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two-lane form of exp2_poly on the packed fp32x2 pipe: the rounding adds, the reduced argument
+// and the three polynomial steps are one FADD2 / FFMA2 each for both lanes; the clamp and the
+// exponent insertion (one integer multiply-add) stay per lane.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  const float2 r = __fadd2_rn(xc, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(r, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), xc);  // xc - n, exact
+  float2 p = __ffma2_rn(make_float2(kExpC3, kExpC3), f, make_float2(kExpC2, kExpC2));
+  p = __ffma2_rn(p, f, make_float2(kExpC1, kExpC1));
+  p = __ffma2_rn(p, f, make_float2(kExpC0, kExpC0));
+  return make_float2(__uint_as_float(__float_as_uint(r.x) * 8388608u + __float_as_uint(p.x)),
+                     __uint_as_float(__float_as_uint(r.y) * 8388608u + __float_as_uint(p.y)));
+}
+
+// Columns [J0, J0 + 64) of one score row, in place: p_j = 2^(s_j * sl2 - base), packed to bf16
+// pairs into r[J0/2, J0/2 + 32) (the scores there are already consumed); the fp32 p_j are added
+// to four running sums. The scale-subtract uses the packed fp32x2 FMA (two columns per
+// instruction); column pairs (j, j+1) with bit (j/2) % 8 of kPolyMask set take exp2_poly2, the
+// rest ex2.approx.
+template <int J0>
+__device__ __forceinline__ void exp_pack_64(uint32_t* r, float2 sc, float2 nb, float2 (&acc)[2]) {
+  const float* s = reinterpret_cast<const float*>(r);
+#pragma unroll
+  for (int j = J0; j < J0 + 64; j += 2) {
+    const float2 x = __ffma2_rn(make_float2(s[j], s[j + 1]), sc, nb);
+    const float2 p = ((kPolyMask >> ((j / 2) & 7)) & 1u) ? exp2_poly2(x) : make_float2(ex2f(x.x), ex2f(x.y));
+    acc[(j / 2) & 1].x += p.x;
+    acc[(j / 2) & 1].y += p.y;
+    r[j / 2] = pack_bf16(p.x, p.y);
+  }
 }
 
 #endif  // __CUDACC__

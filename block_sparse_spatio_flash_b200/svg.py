@@ -76,7 +76,7 @@ _sig = {
     "svg_dense_attention_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _i32,
                                                _vp, _sz, _vp, _vp]),
     "svg_read_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int32), _vp]),
-    "svg_route_work_bytes": (_sz, [_i32, _i32]),
+    "svg_route_work_bytes": (_sz, [_i32, _i64, _i32, _i32]),
     "svg_route_heads": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, svg_geom, svg_mask, _vp, _i32,
                                        _vp, _sz, _vp, _vp, _vp]),
     "svg_attention_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p,
@@ -211,8 +211,8 @@ def svg_attention_fwd_noalloc(q, k, v, o, routes, ws_spatial, ws_temporal, geom,
     return o
 
 
-def svg_route_work_bytes(heads: int, n_rows: int) -> int:
-    return int(_lib.svg_route_work_bytes(heads, n_rows))
+def svg_route_work_bytes(heads: int, tokens: int, d: int, n_rows: int) -> int:
+    return int(_lib.svg_route_work_bytes(heads, tokens, d, n_rows))
 
 
 def svg_route_heads(q, k, v, geom, mask, rows, route, err=None, work=None, scale: float = 0.0,
@@ -221,7 +221,7 @@ def svg_route_heads(q, k, v, geom, mask, rows, route, err=None, work=None, scale
     q/k/v [H, N, d] bf16 original order, rows int32, route uint8 [H], err float32 [H, 2])."""
     heads, tokens, d = q.shape
     if work is None:
-        work = torch.empty(svg_route_work_bytes(heads, rows.numel()), dtype=torch.uint8, device=q.device)
+        work = torch.empty(svg_route_work_bytes(heads, tokens, d, rows.numel()), dtype=torch.uint8, device=q.device)
     _check(_lib.svg_route_heads(_ptr(q), _ptr(k), _ptr(v), heads, tokens, d, scale, geom, mask, _ptr(rows),
                                 rows.numel(), _ptr(work), work.numel() * work.element_size(), _ptr(route),
                                 _ptr(err), _stream(stream)), "svg_route_heads")

@@ -220,11 +220,14 @@ int svg_attention_fwd_noalloc(const void *q, const void *k, const void *v, void 
  *   d_err[2h], d_err[2h+1] = E_spatial / E_d, E_temporal / E_d   (d_err nullable)
  *   q, k, v:  [heads, tokens, d] bf16 in ORIGINAL order (before any permutation).
  *   d_rows:   device int32 [n_rows]; entries outside [0, tokens) are ignored.
- *   d_work:   device buffer of svg_route_work_bytes(heads, n_rows) bytes (per-row errors).
+ *   d_work:   device buffer of svg_route_work_bytes(heads, tokens, d, n_rows) bytes, 4-byte
+ *             aligned (per-row errors, and the softmax state of each key chunk of each row).
  *   d_route:  device uint8 [heads].
  * The sums over rows run in a fixed order, so the decision is deterministic.
+ * Errors: SVG_ERR_ARG (null or misaligned pointer, bad geometry/mask, tokens != frames*H*W),
+ *   SVG_ERR_UNSUPPORTED (d not 64 or 128), SVG_ERR_WORKSPACE (work_bytes too small), SVG_ERR_CUDA.
  */
-size_t svg_route_work_bytes(int32_t heads, int32_t n_rows);
+size_t svg_route_work_bytes(int32_t heads, int64_t tokens, int32_t d, int32_t n_rows);
 int svg_route_heads(const void *q, const void *k, const void *v, int32_t heads, int64_t tokens,
                     int32_t d, float scale, svg_geom geom, svg_mask mask, const int32_t *d_rows,
                     int32_t n_rows, void *d_work, size_t work_bytes, uint8_t *d_route,

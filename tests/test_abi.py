@@ -120,3 +120,28 @@ def test_permute_argument_checks(svg):
     assert f(a, b, 2, 512, 64, routes, g, m, 2, None) == -1           # inverse flag
     bad = (ctypes.c_uint8 * 2)(0, 7)
     assert f(a, b, 2, 512, 64, bad, g, m, 0, None) == -1              # route value
+
+
+def test_route_argument_checks(svg):
+    """Head routing: workspace size and argument rejections, all before any device work."""
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    g, m = svg.make_geom(4, 8, 16), svg.make_mask(1, 16)
+    wb = svg.svg_route_work_bytes
+    assert wb(2, 512, 64, 0) == 0 and wb(0, 512, 64, 8) == 0 and wb(2, 512, 96, 8) == 0
+    # per-row errors (rounded to 256 bytes) + one chunk state of 3 x (d + 2) floats per row
+    assert wb(2, 512, 64, 8) == 256 + 2 * 8 * 1 * 3 * 66 * 4
+    # 75,600 keys: 37 chunks of 2,048 would exceed the cap of 32
+    assert wb(10, 75600, 128, 64) == (10 * 64 * 3 * 4 + 255) // 256 * 256 + 10 * 64 * 32 * 3 * 130 * 4
+    f = lib.svg_route_heads
+    f.argtypes = svg._sig["svg_route_heads"][1]
+    p, rt = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 24)
+    ok_bytes = wb(2, 512, 64, 8)
+    assert f(None, p, p, 2, 512, 64, 0.0, g, m, p, 8, p, ok_bytes, rt, None, None) == -1       # null q
+    assert f(p, p, p, 2, 512, 64, 0.0, g, m, None, 8, p, ok_bytes, rt, None, None) == -1       # null rows
+    assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 8, p, ok_bytes, None, None, None) == -1        # null route
+    assert f(ctypes.c_void_p((1 << 20) + 8), p, p, 2, 512, 64, 0.0, g, m, p, 8, p, ok_bytes, rt, None,
+             None) == -1                                                                    # misaligned q
+    assert f(p, p, p, 2, 511, 64, 0.0, g, m, p, 8, p, ok_bytes, rt, None, None) == -1         # tokens mismatch
+    assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 0, p, ok_bytes, rt, None, None) == -1         # no rows
+    assert f(p, p, p, 2, 512, 96, 0.0, g, m, p, 8, p, ok_bytes, rt, None, None) == -2         # d
+    assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 8, p, ok_bytes - 4, rt, None, None) == -5     # workspace

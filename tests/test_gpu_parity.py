@@ -254,6 +254,25 @@ def test_rounded_row_without_keys_gives_zero(S):
     assert stats
 
 
+@pytest.mark.parametrize("dense", [False, True])
+@pytest.mark.parametrize("bk", [64, 128])
+def test_attention_growing_maxima(S, dense, bk):
+    """Keys planted at random positions with scores up to ~9x the others: a row's running maximum
+    jumps past the rescale threshold in the middle of the row, which exercises the redo of a tile
+    whose exponentials were taken against the old maximum, and the O correction."""
+    w = MEDIUM.replace(bk=bk)
+    q, k, v = syn.make_qkv(w, seed_offset=13)
+    k = k.float()
+    g = torch.Generator().manual_seed(77)
+    for h in range(w.heads):
+        idx = torch.randperm(w.tokens, generator=g)[:24]
+        k[h, idx] *= torch.linspace(2.0, 9.0, 24)[:, None]
+    k = k.to(torch.bfloat16)
+    out, lse, st = gp.run_path(w, q, k, v, dense=dense, bk=bk)
+    assert st == 0
+    gp.compare_rows(w, q, k, v, out, lse, all_kept=dense)
+
+
 def test_naive_equals_split_up_to_rounding(S):
     w = MEDIUM
     q, k, v = syn.make_qkv(w, seed_offset=7)
@@ -360,3 +379,15 @@ def test_route_pages_shape(S):
     got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
     _check_routes(got_r, got_e, want_r, want_e)
     assert list(got_r) == kinds
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_route_several_key_chunks(S, d):
+    """4,620 keys: three key chunks of 1,600 (the last ragged), 100 sampled rows (a ragged row block)."""
+    w = syn.Workload("route_chunks", frames=7, grid_h=20, grid_w=33, routes=(1, 0, 1), d=d,
+                     frame_window=1, spatial_band=40)
+    q, k, v = syn.make_routed_qkv(w, list(w.routes), strength=1.2, seed_offset=9)
+    rows = np.sort(np.random.default_rng(5).choice(w.tokens, 100, replace=False))
+    got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
+    _check_routes(got_r, got_e, want_r, want_e)
+    assert list(got_r) == list(w.routes)
