@@ -424,6 +424,169 @@ int svg_route_heads(const void* q, const void* k, const void* v, int32_t heads, 
                       static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------------------
+// Host-buffer entry point: chunks of heads flow through three library streams (copies in,
+// compute, copies out) and two device slots, so the copies of one chunk overlap the
+// permutation and attention of the neighbouring chunks.
+namespace {
+
+struct HostPipe {
+  cudaStream_t in, comp, out;
+  cudaEvent_t h2d[2], done[2], d2h[2];
+  std::mutex call;  // one host-buffer call per device at a time: the streams and events are shared
+};
+
+HostPipe* host_pipe(int* rc) {
+  static std::mutex mu;
+  static HostPipe* pipes[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *rc = SVG_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pipes[dev]) {
+    HostPipe* hp = new HostPipe();
+    cudaError_t e = cudaStreamCreateWithFlags(&hp->in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp->comp, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp->out, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&hp->h2d[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp->done[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp->d2h[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) {  // the partly built pipe is kept out of use (and leaked) on this path
+      *rc = record_cuda_error("host pipe streams / events", e);
+      return nullptr;
+    }
+    pipes[dev] = hp;
+  }
+  return pipes[dev];
+}
+
+size_t chunk_tensor_bytes(int64_t tokens, int d, int chunk_heads) {
+  return ((size_t)chunk_heads * tokens * d * 2 + 255) / 256 * 256;
+}
+
+// Keeps the first nonzero status of the chunks' attention launches (each launch clears its own).
+__global__ void keep_status(const int* launch_status, int* call_status) {
+  const int v = *launch_status;
+  if (v != 0 && *call_status == 0) *call_status = v;
+}
+
+}  // namespace
+
+size_t svg_attention_host_buffer_bytes(int64_t tokens, int32_t d, int32_t chunk_heads) {
+  if (tokens < 1 || tokens > kMaxTokens || (d != 64 && d != 128) || chunk_heads < 1 || chunk_heads > kMaxHeads)
+    return 0;
+  return 2 * 7 * chunk_tensor_bytes(tokens, d, chunk_heads) + kScratchBytes + 256;
+}
+
+int svg_attention_fwd_host(const void* h_q, const void* h_k, const void* h_v, void* h_o, int32_t heads,
+                           int64_t tokens, int32_t d, float scale, const uint8_t* h_route,
+                           const void* d_ws_spatial, const void* d_ws_temporal, svg_geom geom, svg_mask mask,
+                           svg_tile tile, int32_t mode, int32_t chunk_heads, void* d_buf, size_t buf_bytes) {
+  if (!h_q || !h_k || !h_v || !h_o || !h_route || !d_buf || !aligned(d_buf, 256)) return SVG_ERR_ARG;
+  if (heads < 1 || heads > kMaxHeads || chunk_heads < 1) return SVG_ERR_ARG;
+  if (!geom_ok(geom) || !mask_ok(geom, mask)) return SVG_ERR_ARG;
+  if ((int64_t)geom.frames * geom.grid_h * geom.grid_w != tokens) return SVG_ERR_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  if (!tile_ok(tile)) return SVG_ERR_UNSUPPORTED;
+  if (mode != SVG_MODE_SPLIT && mode != SVG_MODE_NAIVE) return SVG_ERR_ARG;
+  for (int h = 0; h < heads; ++h)
+    if (h_route[h] > 1) return SVG_ERR_ARG;
+  const int ch = chunk_heads < heads ? chunk_heads : heads;
+  if (buf_bytes < svg_attention_host_buffer_bytes(tokens, d, ch)) return SVG_ERR_WORKSPACE;
+  int num_sms = 0;
+  int rc = device_info(&num_sms);
+  if (rc) return rc;
+  HostPipe* hp = host_pipe(&rc);
+  if (!hp) return rc;
+  std::lock_guard<std::mutex> lock(hp->call);
+
+  const size_t ta = chunk_tensor_bytes(tokens, d, ch);
+  uint8_t* buf = static_cast<uint8_t*>(d_buf);
+  void* scratch = buf + 2 * 7 * ta;
+  int* call_status = reinterpret_cast<int*>(buf + 2 * 7 * ta + kScratchBytes);
+  const size_t head_bytes = (size_t)tokens * d * 2;
+  const int nchunks = (heads + ch - 1) / ch;
+  cudaError_t e = cudaSuccess;
+  const char* what = "";
+#define SVG_HOST_TRY(call, name) \
+  do {                           \
+    e = (call);                  \
+    if (e != cudaSuccess) {      \
+      what = name;               \
+      goto fail;                 \
+    }                            \
+  } while (0)
+  SVG_HOST_TRY(cudaMemsetAsync(call_status, 0, sizeof(int), hp->comp), "cudaMemsetAsync(status)");
+  for (int c = 0; c < nchunks; ++c) {
+    const int h0 = c * ch, hn = (heads - h0) < ch ? (heads - h0) : ch;
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hn * head_bytes;
+    const int s = c & 1;
+    uint8_t* base = buf + (size_t)s * 7 * ta;
+    uint8_t *qo = base, *ko = base + ta, *vo = base + 2 * ta;
+    uint8_t *qp = base + 3 * ta, *kp = base + 4 * ta, *vp = base + 5 * ta, *op = base + 6 * ta;
+    const uint8_t* routes = h_route + h0;
+    bool perm = false;
+    for (int h = 0; h < hn; ++h) perm |= routes[h] != 0;
+    // copies in: the slot's previous chunk must have left the device (its copy out read qo or op)
+    if (c >= 2) SVG_HOST_TRY(cudaStreamWaitEvent(hp->in, hp->d2h[s], 0), "cudaStreamWaitEvent(in)");
+    SVG_HOST_TRY(cudaMemcpyAsync(qo, static_cast<const uint8_t*>(h_q) + off, bytes, cudaMemcpyHostToDevice, hp->in),
+                 "cudaMemcpyAsync(q in)");
+    SVG_HOST_TRY(cudaMemcpyAsync(ko, static_cast<const uint8_t*>(h_k) + off, bytes, cudaMemcpyHostToDevice, hp->in),
+                 "cudaMemcpyAsync(k in)");
+    SVG_HOST_TRY(cudaMemcpyAsync(vo, static_cast<const uint8_t*>(h_v) + off, bytes, cudaMemcpyHostToDevice, hp->in),
+                 "cudaMemcpyAsync(v in)");
+    SVG_HOST_TRY(cudaEventRecord(hp->h2d[s], hp->in), "cudaEventRecord(h2d)");
+    // compute: temporal heads to their order, attention, O back to the original order
+    SVG_HOST_TRY(cudaStreamWaitEvent(hp->comp, hp->h2d[s], 0), "cudaStreamWaitEvent(comp)");
+    if (perm) {
+      if ((rc = launch_permute(qo, qp, hn, tokens, d, routes, geom, mask, 0, num_sms, hp->comp)) ||
+          (rc = launch_permute(ko, kp, hn, tokens, d, routes, geom, mask, 0, num_sms, hp->comp)) ||
+          (rc = launch_permute(vo, vp, hn, tokens, d, routes, geom, mask, 0, num_sms, hp->comp)))
+        goto fail_rc;
+      rc = run_attention(qp, kp, vp, op, nullptr, hn, tokens, d, scale, routes, d_ws_spatial, d_ws_temporal, &geom,
+                         &mask, tile.bq, tile.bk, mode, false, scratch, kScratchBytes, nullptr, hp->comp);
+      if (rc) goto fail_rc;
+      if ((rc = launch_permute(op, qo, hn, tokens, d, routes, geom, mask, 1, num_sms, hp->comp))) goto fail_rc;
+    } else {
+      rc = run_attention(qo, ko, vo, op, nullptr, hn, tokens, d, scale, routes, d_ws_spatial, d_ws_temporal, &geom,
+                         &mask, tile.bq, tile.bk, mode, false, scratch, kScratchBytes, nullptr, hp->comp);
+      if (rc) goto fail_rc;
+    }
+    keep_status<<<1, 1, 0, hp->comp>>>(static_cast<const int*>(scratch), call_status);
+    SVG_HOST_TRY(cudaGetLastError(), "launch keep_status");
+    SVG_HOST_TRY(cudaEventRecord(hp->done[s], hp->comp), "cudaEventRecord(done)");
+    // copy out
+    SVG_HOST_TRY(cudaStreamWaitEvent(hp->out, hp->done[s], 0), "cudaStreamWaitEvent(out)");
+    SVG_HOST_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(h_o) + off, perm ? qo : op, bytes, cudaMemcpyDeviceToHost,
+                                 hp->out),
+                 "cudaMemcpyAsync(o out)");
+    SVG_HOST_TRY(cudaEventRecord(hp->d2h[s], hp->out), "cudaEventRecord(d2h)");
+  }
+#undef SVG_HOST_TRY
+  {
+    e = cudaStreamSynchronize(hp->out);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(hp->comp);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(hp->in);
+    if (e != cudaSuccess) return record_cuda_error("cudaStreamSynchronize(host pipe)", e);
+    int32_t st = 0;
+    e = cudaMemcpy(&st, call_status, sizeof(st), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return record_cuda_error("cudaMemcpy(status)", e);
+    return st;
+  }
+fail:
+  rc = record_cuda_error(what, e);
+fail_rc:
+  // let whatever was queued finish before the caller may free or reuse its buffers
+  cudaStreamSynchronize(hp->out);
+  cudaStreamSynchronize(hp->comp);
+  cudaStreamSynchronize(hp->in);
+  return rc;
+}
+
 int svg_read_status(const void* d_scratch_or_status, int32_t* h_status, void* stream) {
   if (!d_scratch_or_status || !h_status || !aligned(d_scratch_or_status, 4)) return SVG_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -81,6 +81,9 @@ _sig = {
                                        _vp, _sz, _vp, _vp, _vp]),
     "svg_attention_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p,
                                                  _vp, _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _vp]),
+    "svg_attention_host_buffer_bytes": (_sz, [_i64, _i32, _i32]),
+    "svg_attention_fwd_host": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp, _vp,
+                                              svg_geom, svg_mask, svg_tile, _i32, _i32, _vp, _sz]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -208,6 +211,31 @@ def svg_attention_fwd_noalloc(q, k, v, o, routes, ws_spatial, ws_temporal, geom,
     _check(_lib.svg_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), heads, tokens, d, scale,
                                           _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile,
                                           mode, _ptr(status), _stream(stream)), "svg_attention_fwd_noalloc")
+    return o
+
+
+def _hptr(t: torch.Tensor):
+    if t.is_cuda:
+        raise ValueError("expected a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def svg_attention_host_buffer_bytes(tokens: int, d: int, chunk_heads: int) -> int:
+    return int(_lib.svg_attention_host_buffer_bytes(tokens, d, chunk_heads))
+
+
+def svg_attention_fwd_host(q, k, v, o, routes, ws_spatial, ws_temporal, geom, mask, tile, buf, chunk_heads=1,
+                           mode=SVG_MODE_SPLIT, scale: float = 0.0) -> torch.Tensor:
+    """End to end on host tensors (q/k/v/o: CPU [H, N, d] bf16, original order; pinned memory
+    overlaps the copies with compute). buf: device uint8 tensor of
+    svg_attention_host_buffer_bytes(N, d, min(chunk_heads, H)) bytes. Synchronous."""
+    heads, tokens, d = q.shape
+    _check(_lib.svg_attention_fwd_host(_hptr(q), _hptr(k), _hptr(v), _hptr(o), heads, tokens, d, scale,
+                                       _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile, mode,
+                                       chunk_heads, _ptr(buf), buf.numel() * buf.element_size()),
+           "svg_attention_fwd_host")
     return o
 
 

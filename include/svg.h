@@ -233,6 +233,35 @@ int svg_route_heads(const void *q, const void *k, const void *v, int32_t heads, 
                     int32_t n_rows, void *d_work, size_t work_bytes, uint8_t *d_route,
                     float *d_err, void *stream);
 
+/*
+ * End-to-end attention on HOST buffers: copies Q/K/V to the device, takes temporal heads to
+ * their token order, runs svg_attention_fwd, takes O back to the original order and copies it
+ * to the host; the same computation as svg_permute + svg_attention_fwd + svg_permute(inverse)
+ * on device buffers, with bitwise-identical results. Heads go through in chunks of
+ * `chunk_heads`, on three streams owned by the library (copies in, compute, copies out) and two
+ * device slots, so that one chunk's copies overlap the neighbouring chunks' compute
+ * ("Sources & evidence" of the case study: the pages time the attention kernel alone and leave
+ * out host transfers; this call is what a user without device buffers runs).
+ *   h_q, h_k, h_v: host [heads, tokens, d] bf16, ORIGINAL order. Page-locked memory
+ *                  (cudaHostAlloc / cudaHostRegister) lets the copies overlap compute; pageable
+ *                  memory works but serialises them.
+ *   h_o:           host [heads, tokens, d] bf16 out, original order.
+ *   h_route, d_ws_spatial, d_ws_temporal, geom, mask, tile, mode: as for svg_attention_fwd.
+ *   chunk_heads:   heads per chunk (>= 1; values above `heads` act as `heads`).
+ *   d_buf:         device buffer, 256-byte aligned, of
+ *                  svg_attention_host_buffer_bytes(tokens, d, min(chunk_heads, heads)) bytes.
+ * Synchronous: returns once h_o holds the result. Calls on one device are serialised (the
+ * streams are shared). Returns SVG_OK, an argument error before any device work, SVG_ERR_CUDA,
+ * or the first device status a chunk reported (SVG_ERR_TIMEOUT / SVG_ERR_WORKSPACE).
+ */
+size_t svg_attention_host_buffer_bytes(int64_t tokens, int32_t d, int32_t chunk_heads);
+int svg_attention_fwd_host(const void *h_q, const void *h_k, const void *h_v, void *h_o,
+                           int32_t heads, int64_t tokens, int32_t d, float scale,
+                           const uint8_t *h_route, const void *d_ws_spatial,
+                           const void *d_ws_temporal, svg_geom geom, svg_mask mask,
+                           svg_tile tile, int32_t mode, int32_t chunk_heads, void *d_buf,
+                           size_t buf_bytes);
+
 /* Reads the device status word of a scratch buffer (or d_status). Synchronises `stream`. */
 int svg_read_status(const void *d_scratch_or_status, int32_t *h_status, void *stream);
 

@@ -145,3 +145,30 @@ def test_route_argument_checks(svg):
     assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 0, p, ok_bytes, rt, None, None) == -1         # no rows
     assert f(p, p, p, 2, 512, 96, 0.0, g, m, p, 8, p, ok_bytes, rt, None, None) == -2         # d
     assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 8, p, ok_bytes - 4, rt, None, None) == -5     # workspace
+
+
+def test_host_entry_argument_checks(svg):
+    """Host-buffer entry point: buffer size rule and rejections before any device work."""
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    hb = svg.svg_attention_host_buffer_bytes
+    one = (512 * 64 * 2 + 255) // 256 * 256
+    assert hb(512, 64, 1) == 2 * 7 * one + 256 + 256
+    assert hb(512, 96, 1) == 0 and hb(512, 64, 0) == 0 and hb(0, 64, 1) == 0
+    f = lib.svg_attention_fwd_host
+    f.argtypes = svg._sig["svg_attention_fwd_host"][1]
+    g, m, t = svg.make_geom(4, 8, 16), svg.make_mask(1, 16), svg.make_tile(64, 64)
+    routes = (ctypes.c_uint8 * 2)(0, 1)
+    hbuf = ctypes.create_string_buffer(16)
+    h = ctypes.cast(hbuf, ctypes.c_void_p)
+    dbuf = ctypes.c_void_p(1 << 20)
+    need = hb(512, 64, 2)
+    assert f(None, h, h, h, 2, 512, 64, 0.0, routes, dbuf, dbuf, g, m, t, 0, 2, dbuf, need) == -1   # null q
+    assert f(h, h, h, h, 2, 512, 64, 0.0, routes, dbuf, dbuf, g, m, t, 0, 0, dbuf, need) == -1      # chunk 0
+    assert f(h, h, h, h, 2, 511, 64, 0.0, routes, dbuf, dbuf, g, m, t, 0, 2, dbuf, need) == -1      # tokens
+    assert f(h, h, h, h, 2, 512, 64, 0.0, routes, dbuf, dbuf, g, m, t, 0, 2,
+             ctypes.c_void_p((1 << 20) + 16), need) == -1                                          # alignment
+    assert f(h, h, h, h, 2, 512, 96, 0.0, routes, dbuf, dbuf, g, m, t, 0, 2, dbuf, need) == -2      # d
+    assert f(h, h, h, h, 2, 512, 64, 0.0, routes, dbuf, dbuf, g, m, t, 7, 2, dbuf, need) == -1      # mode
+    assert f(h, h, h, h, 2, 512, 64, 0.0, routes, dbuf, dbuf, g, m, t, 0, 2, dbuf, need - 1) == -5  # buffer
+    bad = (ctypes.c_uint8 * 2)(0, 3)
+    assert f(h, h, h, h, 2, 512, 64, 0.0, bad, dbuf, dbuf, g, m, t, 0, 2, dbuf, need) == -1         # route

@@ -391,3 +391,24 @@ def test_route_several_key_chunks(S, d):
     got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
     _check_routes(got_r, got_e, want_r, want_e)
     assert list(got_r) == list(w.routes)
+
+
+# ----------------------------------------------------------------------------- host-buffer entry
+@pytest.mark.parametrize("chunk", [1, 3, 4, 9])
+@pytest.mark.parametrize("routes", [(0, 1, 0, 1), (0, 0, 0, 0), (1, 1, 0, 1)])
+def test_host_entry_matches_device_path(S, chunk, routes):
+    """svg_attention_fwd_host (pinned host buffers, chunked pipeline) gives exactly the bytes of
+    the device-buffer path, and so the oracle's values."""
+    w = MEDIUM.replace(routes=routes)
+    q, k, v = syn.make_qkv(w, seed_offset=17)
+    want, lse, st = gp.run_path(w, q, k, v)
+    assert st == 0
+    g, m, t = gp.geom_mask_tile(w)
+    maps = gp.build_maps(w, g, m, t, list(routes))
+    qh, kh, vh = (x.contiguous().pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    buf = torch.empty(S.svg_attention_host_buffer_bytes(w.tokens, w.d, min(chunk, w.heads)), dtype=torch.uint8,
+                      device="cuda")
+    S.svg_attention_fwd_host(qh, kh, vh, oh, list(routes), maps[0], maps[1], g, m, t, buf, chunk_heads=chunk)
+    assert torch.equal(oh.view(torch.int16), want.view(torch.int16))
+    gp.compare_rows(w, q, k, v, oh, None)
