@@ -113,6 +113,25 @@ int encode_qkv_map(CUtensorMap* m, const void* base, int heads, int tokens, int 
   return SVG_OK;
 }
 
+// [heads * tokens, d] bf16 viewed as rows, box 64 columns x 1 row, 128-byte swizzle: the map
+// for 4-row gathers of arbitrary rows.
+int encode_rows_map(CUtensorMap* m, const void* base, int heads, int64_t tokens, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return record_cuda_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", (int)cudaErrorSymbolNotFound);
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)tokens * heads};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (rows): CUresult %d", (int)r);
+    return SVG_ERR_CUDA;
+  }
+  return SVG_OK;
+}
+
 // The single-SM kernel serves every call; SVG_KERNEL=pair in the environment (read once)
 // selects the SM-pair kernel (two-SM MMAs, each SM loading half of every K/V tile) for d = 128,
 // to compare the two.
@@ -137,7 +156,7 @@ int check_qkvo(const void* q, const void* k, const void* v, const void* o, const
 int run_attention(const void* q, const void* k, const void* v, void* o, float* lse, int heads, int64_t tokens,
                   int d, float scale, const uint8_t* h_route, const void* ws_sp, const void* ws_tm,
                   const svg_geom* geom, const svg_mask* mask, int bq, int bk, int mode, bool dense,
-                  void* scratch, size_t scratch_bytes, int32_t* d_status, cudaStream_t st) {
+                  void* scratch, size_t scratch_bytes, int32_t* d_status, cudaStream_t st, bool fused = false) {
   int rc = check_qkvo(q, k, v, o, lse, heads, tokens, d);
   if (rc) return rc;
   if (!scratch || scratch_bytes < kScratchBytes || !aligned(scratch, 16)) return SVG_ERR_ARG;
@@ -152,7 +171,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   std::lock_guard<std::mutex> lock(mu);
   memset(&P, 0, sizeof(P));
   const int N = (int)tokens;
-  const bool pair = use_pair_kernel(d);
+  const bool pair = use_pair_kernel(d) && !fused;
   P.H = heads;
   P.N = N;
   P.nk = (N + bk - 1) / bk;
@@ -166,6 +185,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   P.dense = dense ? 1 : 0;
   P.bkm = bk;
   P.naive = mode == SVG_MODE_NAIVE ? 1 : 0;
+  P.fused = fused && !dense ? 1 : 0;
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
   P.status = d_status ? d_status : static_cast<int*>(scratch);
@@ -218,6 +238,11 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
   if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, pair ? bk / 2 : bk))) return rc;
   if ((rc = encode_qkv_map(&P.tm_v, v, heads, N, d, bk))) return rc;
+  if (P.fused && P.uses[SVG_ROUTE_TEMPORAL]) {
+    if ((rc = encode_rows_map(&P.tm_q2, q, heads, N, d))) return rc;
+    if ((rc = encode_rows_map(&P.tm_k2, k, heads, N, d))) return rc;
+    if ((rc = encode_rows_map(&P.tm_v2, v, heads, N, d))) return rc;
+  }
   cudaError_t me = cudaMemsetAsync(scratch, 0, kScratchBytes, st);
   if (me == cudaSuccess && d_status) me = cudaMemsetAsync(d_status, 0, sizeof(int32_t), st);
   if (me != cudaSuccess) return record_cuda_error("cudaMemsetAsync(scratch)", me);
@@ -378,6 +403,15 @@ int svg_attention_fwd(const void* q, const void* k, const void* v, void* o, floa
   return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
                        tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
                        static_cast<cudaStream_t>(stream));
+}
+
+int svg_attention_fwd_fused(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,
+                            int64_t tokens, int32_t d, float scale, const uint8_t* h_route, const void* d_ws_spatial,
+                            const void* d_ws_temporal, svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
+                            void* d_scratch, size_t scratch_bytes, int32_t* d_status, void* stream) {
+  return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
+                       tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
+                       static_cast<cudaStream_t>(stream), true);
 }
 
 int svg_dense_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,

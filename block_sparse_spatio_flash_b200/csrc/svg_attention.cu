@@ -339,60 +339,92 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 
   if (!skip_all && warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t kv_pos = 0, q_iter = 0;
-      bool q_issued = false;
-      for (uint32_t it = 0;; ++it) {
-        const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
-        if (!wait_bar(c.item_empty(slot), ph ^ 1u, abort_addr, status)) break;
-        const uint32_t idx = atomicAdd(P.counter, 1u);
-        const ItemInfo inf = decode_item<BK>(P, idx);
+    // Lane 0 takes the waits, the work counter and the transaction counts; the results are
+    // broadcast so that the whole warp follows the same control flow. Tiled loads are issued by
+    // lane 0; in fused token order a temporal item's rows are gathered, lane L fetching rows
+    // 4L .. 4L + 3 of each tile (their original indices) for both 64-column chunks.
+    uint32_t kv_pos = 0, q_iter = 0;
+    bool q_issued = false;
+    for (uint32_t it = 0;; ++it) {
+      const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
+      if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.item_empty(slot), ph ^ 1u, abort_addr, status) : 0,
+                       0))
+        break;
+      const uint32_t idx = __shfl_sync(0xffffffffu, lane == 0 ? atomicAdd(P.counter, 1u) : 0u, 0);
+      const ItemInfo inf = decode_item<BK>(P, idx);
+      if (lane == 0) {
         items[slot] = inf;
         mbar_arrive(c.item_full(slot));
-        if (!inf.valid) break;
-        if (inf.nA + inf.nB > 0) {
-          if (!wait_bar(c.q_free(), (q_iter & 1u) ^ 1u, abort_addr, status)) break;
-          ++q_iter;
-          const uint32_t bytes = (uint32_t)C::kQHalfBytes * ((inf.nA > 0) + (inf.nB > 0));
-          mbar_expect_tx(c.q_full(), bytes);
-          for (int h = 0; h < 2; ++h) {
-            if ((h == 0 ? inf.nA : inf.nB) == 0) continue;
+      }
+      if (!inf.valid) break;
+      const bool gat = P.fused && inf.cls == SVG_ROUTE_TEMPORAL;
+      const MaskGeom& gg = P.g[SVG_ROUTE_TEMPORAL];
+      const int hrow = inf.head * P.N;  // first row of the head in the 2-D maps
+      if (inf.nA + inf.nB > 0) {
+        if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.q_free(), (q_iter & 1u) ^ 1u, abort_addr, status) : 0,
+                         0))
+          break;
+        ++q_iter;
+        if (lane == 0) mbar_expect_tx(c.q_full(), (uint32_t)C::kQHalfBytes * ((inf.nA > 0) + (inf.nB > 0)));
+        __syncwarp();
+        for (int h = 0; h < 2; ++h) {
+          if ((h == 0 ? inf.nA : inf.nB) == 0) continue;
+          const int p0 = inf.pair * kPairRows + h * kHalfRows;
+          if (gat) {
+            int rr[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rr[i] = hrow + orig_index(gg, min(p0 + 4 * lane + i, P.N - 1));
             for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_3d(sQ + h * C::kQHalfBytes + ch * (128 * 128), &P.tm_q, c.q_full(), ch * 64,
-                          inf.pair * kPairRows + h * kHalfRows, inf.head);
-          }
-          q_issued = true;
-        }
-        bool ok = true;
-        for (int e = 0; e < inf.count && ok; ++e) {
-          const uint32_t ent = get_entry<BK>(P, inf, e);
-          const int row0 = (int)ent_kt(ent) * BK;
-          for (int w = 0; w < 2; ++w) {
-            const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
-            if (!wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status)) {
-              ok = false;
-              break;
-            }
-            mbar_expect_tx(c.kv_full(st), C::kTileBytes);
-            const uint32_t dst = sRing + st * C::kTileBytes;
+              tma_gather4(sQ + h * C::kQHalfBytes + ch * (128 * 128) + lane * 512, &P.tm_q2, c.q_full(), ch * 64, rr[0],
+                          rr[1], rr[2], rr[3]);
+          } else if (lane == 0) {
             for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_3d(dst + ch * (BK * 128), w == 0 ? &P.tm_k : &P.tm_v, c.kv_full(st), ch * 64, row0,
-                          inf.head);
-            ++kv_pos;
+              tma_load_3d(sQ + h * C::kQHalfBytes + ch * (128 * 128), &P.tm_q, c.q_full(), ch * 64, p0, inf.head);
           }
         }
-        if (!ok) break;
+        q_issued = true;
       }
-      if (ld_shared_volatile(abort_addr)) {  // let issued copies land before the CTA may exit
-        const uint32_t n = kv_pos < (uint32_t)NS ? kv_pos : (uint32_t)NS;
-        for (uint32_t i = 0; i < n; ++i) {
-          const uint32_t pos = kv_pos - 1 - i;
-          drain_bar(c.kv_full(pos % NS), (pos / NS) & 1u);
+      bool ok = true;
+      for (int e = 0; e < inf.count && ok; ++e) {
+        const uint32_t ent = get_entry<BK>(P, inf, e);
+        const int row0 = (int)ent_kt(ent) * BK;
+        int rr[4] = {0, 0, 0, 0};
+        if (gat && 4 * lane < BK) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) rr[i] = hrow + orig_index(gg, min(row0 + 4 * lane + i, P.N - 1));
         }
-        if (q_issued) drain_bar(c.q_full(), (q_iter - 1) & 1u);
+        for (int w = 0; w < 2; ++w) {
+          const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
+          if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status) : 0,
+                           0)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_expect_tx(c.kv_full(st), C::kTileBytes);
+          __syncwarp();
+          const uint32_t dst = sRing + st * C::kTileBytes;
+          if (gat) {
+            if (4 * lane < BK)
+              for (int ch = 0; ch < C::kChunks; ++ch)
+                tma_gather4(dst + ch * (BK * 128) + lane * 512, w == 0 ? &P.tm_k2 : &P.tm_v2, c.kv_full(st), ch * 64,
+                            rr[0], rr[1], rr[2], rr[3]);
+          } else if (lane == 0) {
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tma_load_3d(dst + ch * (BK * 128), w == 0 ? &P.tm_k : &P.tm_v, c.kv_full(st), ch * 64, row0, inf.head);
+          }
+          ++kv_pos;
+        }
       }
+      if (!ok) break;
     }
-    __syncwarp();
+    if (lane == 0 && ld_shared_volatile(abort_addr)) {  // let issued copies land before the CTA may exit
+      const uint32_t n = kv_pos < (uint32_t)NS ? kv_pos : (uint32_t)NS;
+      for (uint32_t i = 0; i < n; ++i) {
+        const uint32_t pos = kv_pos - 1 - i;
+        drain_bar(c.kv_full(pos % NS), (pos / NS) & 1u);
+      }
+      if (q_issued) drain_bar(c.q_full(), (q_iter - 1) & 1u);
+    }
   } else if (!skip_all && warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -509,16 +541,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       const int row = inf.pair * kPairRows + h * kHalfRows + lr;
       const bool in_range = row < P.N;
       const int nmine = h == 0 ? inf.nA : inf.nB;
+      const int prow = in_range ? row : P.N - 1;
+      // where the row lives in Q / O / LSE: its position, or its original index in fused order
+      const int orow_idx = (P.fused && inf.cls == SVG_ROUTE_TEMPORAL) ? orig_index(P.g[SVG_ROUTE_TEMPORAL], prow) : prow;
       if (nmine == 0) {  // no kept key for any row of this half (rounded masks only)
         if (in_range) {
-          __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + row) * D;
+          __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + orow_idx) * D;
           const uint4 z = make_uint4(0, 0, 0, 0);
           for (int x = 0; x < D / 8; ++x) reinterpret_cast<uint4*>(orow)[x] = z;
-          if (P.lse) P.lse[(size_t)inf.head * P.N + row] = -INFINITY;
+          if (P.lse) P.lse[(size_t)inf.head * P.N + orow_idx] = -INFINITY;
         }
         continue;
       }
-      const int prow = in_range ? row : P.N - 1;
       // kept keys of this row: [0, se) U [lo, hi) U (periodic sink), see svg_common.cuh
       int lo = 0, hi = 0, se = 0;
       bool per = false;
@@ -577,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       ++od_cnt;
       tc_fence_after();
       const float inv_l = (l > 0.f && m != -INFINITY) ? 1.f / l : 0.f;  // a row with no kept key gives 0
-      __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + prow) * D;
+      __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + orow_idx) * D;
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
         uint32_t o[32];
@@ -600,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       tc_fence_before();
       mbar_arrive(c.o_free(h));
       if (in_range && P.lse)
-        P.lse[(size_t)inf.head * P.N + row] =
+        P.lse[(size_t)inf.head * P.N + orow_idx] =
             (l > 0.f && m != -INFINITY) ? (m * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }

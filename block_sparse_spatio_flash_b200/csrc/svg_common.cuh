@@ -83,6 +83,13 @@ __host__ __device__ inline void pos_to_ts(const MaskGeom& g, int p, int& t, int&
 }
 
 // Position of token (t, s) in this head's order.
+// Original (frame-major) index of the token at position p of the head's order.
+__host__ __device__ inline int orig_index(const MaskGeom& g, int p) {
+  int t, s;
+  pos_to_ts(g, p, t, s);
+  return t * g.S + s;
+}
+
 __host__ __device__ inline int ts_to_pos(const MaskGeom& g, int t, int s) {
   if (g.route == SVG_ROUTE_SPATIAL) return t * g.S + s;
   if (g.layout == SVG_LAYOUT_FULL_SPACE_MAJOR) return s * g.T + t;
@@ -199,6 +206,11 @@ constexpr size_t kScratchBytes = 256;
 // Launch parameters of the attention kernel (filled on the host, read on the device).
 struct AttnParams {
   CUtensorMap tm_q, tm_k, tm_v;
+  // Fused token order (fused = 1): Q/K/V/O stay in the original order; temporal heads read
+  // their rows with 4-row gathers through these 2-D maps ([heads * N] rows x d, box 64 x 1)
+  // and write O rows back to their original index.
+  CUtensorMap tm_q2, tm_k2, tm_v2;
+  int fused;
   __nv_bfloat16* o;
   float* lse;
   int H, N, npairs, nk, n_items;
@@ -284,6 +296,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// Four rows r0..r3 (any order, any rows) of 64 columns starting at column c0 of a 2-D tensor
+// map with a one-row box, to 4 x 128 bytes at dst (128-byte swizzle as a tiled load of those
+// rows would place them).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int r0, int r1,
+                                            int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

@@ -262,6 +262,23 @@ int svg_attention_fwd_host(const void *h_q, const void *h_k, const void *h_v, vo
                            svg_tile tile, int32_t mode, int32_t chunk_heads, void *d_buf,
                            size_t buf_bytes);
 
+/*
+ * svg_attention_fwd with the token permutation fused into the kernel: q, k, v, o (and lse) are
+ * all in the ORIGINAL frame-major order for every head, and no svg_permute pass is needed. The
+ * pages' kernel runs temporal heads on permuted tokens and leaves the reordering out of its
+ * timings ("routing, token permutation" excluded, "Sources & evidence"); here temporal heads
+ * read each K/V/Q tile's rows where they lie (4-row TMA gathers at their original indices) and
+ * write each O row back to its original index, so the arithmetic, tile by tile, is that of
+ * svg_permute + svg_attention_fwd + svg_permute(inverse) and the results are bitwise equal.
+ * Arguments as svg_attention_fwd; lse (nullable) is [heads, tokens] in original order.
+ */
+int svg_attention_fwd_fused(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int32_t heads, int64_t tokens, int32_t d, float scale,
+                            const uint8_t *h_route, const void *d_ws_spatial,
+                            const void *d_ws_temporal, svg_geom geom, svg_mask mask,
+                            svg_tile tile, int32_t mode, void *d_scratch, size_t scratch_bytes,
+                            int32_t *d_status, void *stream);
+
 /* Reads the device status word of a scratch buffer (or d_status). Synchronises `stream`. */
 int svg_read_status(const void *d_scratch_or_status, int32_t *h_status, void *stream);
 

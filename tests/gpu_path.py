@@ -140,3 +140,30 @@ def tail_rows(w, h, extra=64):
 
 def scale_for(d):
     return 1.0 / math.sqrt(d)
+
+
+def run_fused(w: syn.Workload, q, k, v, *, mode=0, variant=None, bq=None, bk=None, lse=True):
+    """svg_attention_fwd_fused on original-order tensors. Returns (O [H, N, d] bf16 CPU, LSE [H, N]
+    fp32 CPU, both in ORIGINAL order, status)."""
+    S = svg()
+    dev = torch.device("cuda")
+    g, m, t = geom_mask_tile(w, variant, bq, bk)
+    routes = list(w.routes)
+    qd, kd, vd = (x.to(dev).contiguous() for x in (q, k, v))
+    o = torch.empty_like(qd)
+    ls = torch.empty(qd.shape[:2], dtype=torch.float32, device=dev) if lse else None
+    scratch = S.alloc_scratch()
+    maps = build_maps(w, g, m, t, routes)
+    S.svg_attention_fwd_fused(qd, kd, vd, o, routes, maps[0], maps[1], g, m, t, mode=mode, scratch=scratch, lse=ls)
+    status = S.svg_read_status(scratch)
+    torch.cuda.synchronize()
+    return o.cpu(), (ls.cpu() if lse else None), status
+
+
+def lse_to_original(w: syn.Workload, lse):
+    """LSE rows from each head's position order to the original order."""
+    out = torch.empty_like(lse)
+    for h in range(w.heads):
+        pi = oracle.perm_table(w.routes[h], w.layout, w.frames, w.frame_size, w.sink_frames)
+        out[h] = lse[h, torch.as_tensor(pi)]
+    return out

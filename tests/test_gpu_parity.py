@@ -412,3 +412,44 @@ def test_host_entry_matches_device_path(S, chunk, routes):
     S.svg_attention_fwd_host(qh, kh, vh, oh, list(routes), maps[0], maps[1], g, m, t, buf, chunk_heads=chunk)
     assert torch.equal(oh.view(torch.int16), want.view(torch.int16))
     gp.compare_rows(w, q, k, v, oh, None)
+
+
+# ----------------------------------------------------------------------------- fused token order
+FUSED_CASES = [
+    (syn.TINY, {}),
+    (MEDIUM, {}),
+    (MEDIUM, {"bq": 256, "bk": 64}),
+    (MEDIUM.replace(variant=1), {}),
+    (syn.Workload("fused_space_major", frames=6, grid_h=8, grid_w=10, routes=(1, 0, 1), d=128, frame_window=1,
+                  spatial_band=5, layout=1), {}),
+    (syn.Workload("fused_two_sinks", frames=7, grid_h=5, grid_w=9, routes=(1, 0), d=128, frame_window=1,
+                  spatial_band=3, sink_frames=2, bq=256, bk=64), {}),
+    (syn.Workload("fused_d64_ragged", frames=5, grid_h=6, grid_w=9, routes=(1, 1, 0), d=64, frame_window=0,
+                  spatial_band=2, bq=64, bk=64), {}),
+]
+
+
+@pytest.mark.parametrize("w,kw", FUSED_CASES, ids=lambda x: getattr(x, "name", str(x)))
+@pytest.mark.parametrize("mode", [0, 1])
+def test_fused_order_equals_permuted_path(S, w, kw, mode):
+    """Q/K/V/O in original order with temporal rows gathered in-kernel: bitwise the same O (and
+    LSE, mapped to original order) as permute + attention + inverse permute, and the oracle's."""
+    q, k, v = syn.make_qkv(w, seed_offset=21)
+    want, want_lse, st = gp.run_path(w, q, k, v, mode=mode, **kw)
+    assert st == 0
+    got, got_lse, st = gp.run_fused(w, q, k, v, mode=mode, **kw)
+    assert st == 0
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    assert torch.equal(got_lse, gp.lse_to_original(w, want_lse))
+    gp.compare_rows(w, q, k, v, got, None, variant=w.variant, bq=kw.get("bq", w.bq), bk=kw.get("bk", w.bk))
+
+
+def test_fused_order_pages_mixed(S):
+    """75,600 tokens, 5 spatial + 5 temporal heads: fused equals the permuted path bit for bit."""
+    w = syn.MIXED_75K
+    q, k, v = syn.make_qkv(w)
+    want, _, st = gp.run_path(w, q, k, v, lse=False)
+    assert st == 0
+    got, _, st = gp.run_fused(w, q, k, v, lse=False)
+    assert st == 0
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
