@@ -350,7 +350,7 @@ def main():
 # spatial_75600 (128 x 128 tiles, split mode), scaled to the launch's heads: traffic grows with the
 # heads processed. Valid only for the kernel sources that were captured (their SHA-256 prefix);
 # after any change to them the field is null until the capture is repeated.
-CAPTURED_TRAFFIC = {"sources_sha256": "f9bae6f0246475ef", "bytes_per_head": 146.244e6 / 2,
+CAPTURED_TRAFFIC = {"sources_sha256": "27d5e4fe873fef98", "bytes_per_head": 146.841e6 / 2,
                     "workload": "spatial_75600", "bq": 128, "bk": 128, "mode": "split"}
 
 
@@ -426,9 +426,43 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
     work = torch.empty(S.svg_route_work_bytes(w.heads, w.tokens, w.d, rows.numel()), dtype=torch.uint8, device=dev)
     out["route_ms"] = time_events(lambda: S.svg_route_heads(q, k, v, g, m, rows, rt, work=work), 5, stream)
     out["route_rows_per_head"] = int(rows.numel())
+    out["workloads"] = other_workloads(S, P, stream, dev)
     st = S.svg_read_status(scratch)
     out["status"] = st
     return out
+
+
+def other_workloads(S, P, stream, dev):
+    """Attention time (split mode, permuted inputs, 128 x 128 tiles) of the other workloads of the
+    pages' shapes: all-temporal and mixed heads at 75,600 tokens, mixed heads at 302,400 (1440p)."""
+    res = {}
+    for w in (syn.TEMPORAL_75K, syn.MIXED_75K, syn.P1440):
+        g = S.make_geom(w.frames, w.grid_h, w.grid_w)
+        m = S.make_mask(w.frame_window, w.spatial_band, w.sink_frames, w.variant, w.layout)
+        t = S.make_tile(w.bq, w.bk)
+        routes = list(w.routes)
+        q, k, v = (x.to(dev) for x in syn.make_qkv(w))
+        qp, kp, vp = (torch.empty_like(q) for _ in range(3))
+        for a, b in ((q, qp), (k, kp), (v, vp)):
+            S.svg_permute(a, b, routes, g, m)
+        del q, k, v
+        o = torch.empty_like(qp)
+        ws, summ = [None, None], {}
+        for c in sorted(set(routes)):
+            ws[c] = S.alloc_workspace(g, t, dev)
+            S.svg_build_tilemap(g, m, t, c, ws[c])
+            summ[c] = S.svg_tilemap_summary(ws[c])
+        sc = S.alloc_scratch(dev)
+        ms = time_events(lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, scratch=sc), 5,
+                         stream)
+        eff, vis, _ = workload_flops(w, summ)
+        res[w.name] = {"ms": ms, "effective_tflops": eff / (ms * 1e-3) / 1e12,
+                       "visited_tflops": vis / (ms * 1e-3) / 1e12,
+                       "visited_frac_of_peak": vis / (ms * 1e-3) / 1e12 / float(P["bf16_tflops"]),
+                       "status": S.svg_read_status(sc)}
+        del qp, kp, vp, o, ws
+        torch.cuda.empty_cache()
+    return res
 
 
 def end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream, args):

@@ -186,6 +186,10 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   P.bkm = bk;
   P.naive = mode == SVG_MODE_NAIVE ? 1 : 0;
   P.fused = fused && !dense ? 1 : 0;
+  {  // test hook, read on every call: SVG_TEST_STALL=1 makes the launch time out on purpose
+    const char* ts = getenv("SVG_TEST_STALL");
+    P.inject_stall = (ts && ts[0] == '1' && !pair) ? 1 : 0;
+  }
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
   P.status = d_status ? d_status : static_cast<int*>(scratch);

@@ -69,6 +69,7 @@ struct ItemInfo {
 //   2NS + 10 + i   item_full[i]  work item published in slot i
 //   2NS + 12 + i   item_empty[i] slot i read by the MMA warp and the 8 softmax warps
 //   2NS + 14       drain         final MMA completion
+//   2NS + 15       never         completed by nothing (test hook: a wait that runs out)
 //   2NS + 16 ...   two ItemInfo slots, TMEM base, abort flag, workspace check
 template <int NS>
 struct Ctl {
@@ -85,6 +86,7 @@ struct Ctl {
   __device__ __forceinline__ uint32_t item_full(uint32_t i) const { return base + 8u * (2 * NS + 10 + i); }
   __device__ __forceinline__ uint32_t item_empty(uint32_t i) const { return base + 8u * (2 * NS + 12 + i); }
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * (2 * NS + 14); }
+  __device__ __forceinline__ uint32_t never() const { return base + 8u * (2 * NS + 15); }
   static constexpr uint32_t kItemsOff = 8u * (2 * NS + 16);  // 2 x 40 bytes
   static constexpr uint32_t kTmemOff = kItemsOff + 96;
   static constexpr uint32_t kAbortOff = kTmemOff + 8;
@@ -305,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       mbar_init(b + 12 + h, 9);    // item_empty
     }
     mbar_init(b + 14, 1);  // drain
+    mbar_init(b + 15, 1);  // never
     *reinterpret_cast<volatile int*>(ctl_gen + K::kAbortOff) = 0;
     // the tile maps must have been built for exactly these parameters
     int bad = 0;
@@ -531,7 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const uint32_t tO = tmem + lane_off + C::o_col(h);
     const float sl2 = P.sl2;
     uint32_t s_cnt = 0, od_cnt = 0;
-    for (uint32_t it = 0;; ++it) {
+    // (test hook) a wait that nothing satisfies: it gives up after the limit, raises the abort
+    // flag and the timeout status, and every role drains and leaves
+    const bool stalled = P.inject_stall && !__all_sync(0xffffffffu, wait_bar(c.never(), 0, abort_addr, status));
+    for (uint32_t it = 0; !stalled; ++it) {
       const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
       if (!__all_sync(0xffffffffu, wait_bar(c.item_full(slot), ph, abort_addr, status))) break;
       const ItemInfo inf = items[slot];

@@ -211,6 +211,9 @@ struct AttnParams {
   // and write O rows back to their original index.
   CUtensorMap tm_q2, tm_k2, tm_v2;
   int fused;
+  // Test hook: the softmax warps first wait on a barrier that nothing completes, so that the
+  // bounded-wait / abort / drain path runs and the launch ends with SVG_ERR_TIMEOUT.
+  int inject_stall;
   __nv_bfloat16* o;
   float* lse;
   int H, N, npairs, nk, n_items;

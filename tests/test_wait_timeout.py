@@ -1,0 +1,31 @@
+"""Failure detection on the GPU without a fault: a launch whose softmax warps wait on a barrier that
+nothing completes (test hook SVG_TEST_STALL=1) must give up after the bounded wait, report
+SVG_ERR_TIMEOUT through the status word, drain its copies and MMAs, free TMEM and return; the next
+launch in the same context must then run normally and match the oracle."""
+import pytest
+
+from block_sparse_spatio_flash_b200 import synthetic as syn
+from tests import gpu_path as gp
+
+pytestmark = pytest.mark.gpu
+
+W = syn.Workload("timeout_1200", frames=5, grid_h=12, grid_w=20, routes=(0, 1), d=128, frame_window=1,
+                 spatial_band=20)
+
+
+@pytest.fixture(scope="module")
+def S():
+    from block_sparse_spatio_flash_b200 import build
+    build.build()
+    return gp.svg()
+
+
+def test_stalled_wait_reports_timeout_and_context_survives(S, monkeypatch):
+    q, k, v = syn.make_qkv(W, seed_offset=31)
+    monkeypatch.setenv("SVG_TEST_STALL", "1")
+    _, _, st = gp.run_path(W, q, k, v)
+    assert st == S.SVG_ERR_TIMEOUT
+    monkeypatch.delenv("SVG_TEST_STALL")
+    out, lse, st = gp.run_path(W, q, k, v)
+    assert st == 0
+    gp.compare_rows(W, q, k, v, out, lse)
