@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libsvgattn.so")
-SOURCES = ["svg_api.cu", "svg_tilemap.cu", "svg_permute.cu", "svg_attention.cu", "svg_attention2.cu", "svg_route.cu"]
+SOURCES = ["svg_api.cu", "svg_tilemap.cu", "svg_permute.cu", "svg_attention.cu", "svg_attention2.cu", "svg_attention3.cu", "svg_route.cu"]
 HEADERS = ["svg_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

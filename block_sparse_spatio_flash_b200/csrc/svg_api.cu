@@ -17,6 +17,7 @@ int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const
                    svg_mask mask, int inverse, int num_sms, cudaStream_t st);
 int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st);
 int launch_attention_pair(const AttnParams& P, int bk, int max_clusters, cudaStream_t st);
+int launch_attention_pair1(const AttnParams& P, int bk, cudaStream_t st);
 size_t route_work_bytes(int heads, int64_t N, int d, int n_rows);
 int launch_route(const void* q, const void* k, const void* v, int heads, int N, int d, float scale, svg_geom geom,
                  svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
@@ -143,6 +144,15 @@ bool use_pair_kernel(int d) {
   return d == 128 && pair;
 }
 
+// SVG_KERNEL=pair1: SM pairs with one 128-row half per SM and double-buffered scores (d = 128).
+bool use_pair1_kernel(int d) {
+  static const bool pair1 = [] {
+    const char* v = getenv("SVG_KERNEL");
+    return v && strcmp(v, "pair1") == 0;
+  }();
+  return d == 128 && pair1;
+}
+
 int check_qkvo(const void* q, const void* k, const void* v, const void* o, const float* lse, int heads,
                int64_t tokens, int d) {
   if (!q || !k || !v || !o) return SVG_ERR_ARG;
@@ -172,6 +182,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   memset(&P, 0, sizeof(P));
   const int N = (int)tokens;
   const bool pair = use_pair_kernel(d) && !fused;
+  const bool pair1 = use_pair1_kernel(d) && !fused && !pair;
   P.H = heads;
   P.N = N;
   P.nk = (N + bk - 1) / bk;
@@ -188,7 +199,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   P.fused = fused && !dense ? 1 : 0;
   {  // test hook, read on every call: SVG_TEST_STALL=1 makes the launch time out on purpose
     const char* ts = getenv("SVG_TEST_STALL");
-    P.inject_stall = (ts && ts[0] == '1' && !pair) ? 1 : 0;
+    P.inject_stall = (ts && ts[0] == '1' && !pair && !pair1) ? 1 : 0;
   }
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
@@ -240,7 +251,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   // TMA boxes: Q 128 rows; one-SM kernel K and V bk rows; SM-pair kernel: each SM loads bk/2
   // keys of K (all 128 dims) and all bk keys of V for 64 of the dims.
   if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
-  if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, pair ? bk / 2 : bk))) return rc;
+  if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, (pair || pair1) ? bk / 2 : bk))) return rc;
   if ((rc = encode_qkv_map(&P.tm_v, v, heads, N, d, bk))) return rc;
   if (P.fused && P.uses[SVG_ROUTE_TEMPORAL]) {
     if ((rc = encode_rows_map(&P.tm_q2, q, heads, N, d))) return rc;
@@ -251,6 +262,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   if (me == cudaSuccess && d_status) me = cudaMemsetAsync(d_status, 0, sizeof(int32_t), st);
   if (me != cudaSuccess) return record_cuda_error("cudaMemsetAsync(scratch)", me);
   if (pair) return launch_attention_pair(P, bk, (int)(P.n_items < num_sms / 2 ? P.n_items : num_sms / 2), st);
+  if (pair1) return launch_attention_pair1(P, bk, st);
   const int grid = (int)(P.n_items < num_sms ? P.n_items : num_sms);
   return launch_attention(P, d, bk, grid, st);
 }

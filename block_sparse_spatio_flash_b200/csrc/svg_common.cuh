@@ -569,6 +569,102 @@ __device__ __forceinline__ void exp_pack_64(uint32_t* r, float2 sc, float2 nb, f
   }
 }
 
+// A row maximum may grow by up to 2^kRescaleLog2 before O and l are rescaled (log2 units).
+constexpr float kRescaleLog2 = 8.0f;
+
+// ---------------------------------------------------------------------------------------
+// Softmax steps of one score row (one thread per query row, BK scores in registers).
+
+// The row's BK fp32 scores from TMEM.
+template <int BK>
+__device__ __forceinline__ void load_scores(uint32_t tS, uint32_t* r) {
+#pragma unroll
+  for (int q = 0; q < BK / 32; ++q) tmem_ld32(tS + q * 32, r + q * 32);
+  tmem_ld_wait();
+#pragma unroll
+  for (int q = 0; q < BK / 32; ++q) tmem_ld_fence32(r + q * 32);
+}
+
+// Sets to -inf the scores the mask drops: boundary tiles element by element (kept keys of the
+// row are [0, se) U [lo, hi), or the periodic sink of the fully space-major order), the ragged
+// key tail, every visited tile in naive mode, and rows without a kept tile under rounded masks.
+template <int BK>
+__device__ __forceinline__ void mask_scores(const AttnParams& P, int cls, uint32_t f, int c0, int prow, uint32_t ent,
+                                            int lo, int hi, int se, bool per, uint32_t* r) {
+  float* s = reinterpret_cast<float*>(r);
+  const bool elem = (f == kFlagMasked) || (P.naive && !P.dense);
+  if (!(elem || f == kFlagBounds)) return;
+  const int nn = P.N - c0;
+  if (!elem) {
+#pragma unroll
+    for (int j = 0; j < BK; ++j)
+      if (j >= nn) s[j] = -INFINITY;
+  } else if (P.variant == SVG_MASK_ROUNDED) {
+    const uint8_t* rcls = P.cls[cls] + (size_t)(prow / P.bq) * P.nk;
+    const bool rowkept = __ldg(rcls + ent_kt(ent)) == 1;
+#pragma unroll
+    for (int j = 0; j < BK; ++j)
+      if (!(rowkept && j < nn)) s[j] = -INFINITY;
+  } else {
+    const int a = lo - c0;
+    const uint32_t w = (uint32_t)(hi - lo);
+    const int sk = se - c0;
+    if (!per) {
+#pragma unroll
+      for (int j = 0; j < BK; ++j) {
+        const bool keep = (j < nn) && ((j < sk) || ((uint32_t)(j - a) < w));
+        if (!keep) s[j] = -INFINITY;
+      }
+    } else {
+      const MaskGeom& g = P.g[cls];
+      int rr = c0 % g.T;
+#pragma unroll
+      for (int j = 0; j < BK; ++j) {
+        const bool keep = (j < nn) && ((rr < g.F0) || ((uint32_t)(j - a) < w));
+        if (!keep) s[j] = -INFINITY;
+        rr = (rr + 1 == g.T) ? 0 : rr + 1;
+      }
+    }
+  }
+}
+
+// Row maximum first, then the rescale decision: the warp rescales (returns true) when any row's
+// maximum grew by more than 2^kRescaleLog2 or had none yet; l is corrected here, O by the
+// caller after P is stored.
+template <int BK>
+__device__ __forceinline__ bool max_first(const uint32_t* r, float sl2, float& m, float& l, float& alpha) {
+  const float* s = reinterpret_cast<const float*>(r);
+  float mx4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mx4[i] = s[i];
+#pragma unroll
+  for (int j = 4; j < BK; j += 4)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(mx4[i], s[j + i]);
+  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  const float m_new = fmaxf(m, mx);
+  const bool need = (m_new > m) && (m == -INFINITY || (m_new - m) * sl2 > kRescaleLog2);
+  const bool rescale = __any_sync(0xffffffffu, need);
+  if (rescale) {
+    alpha = (m_new == -INFINITY) ? 1.f : ex2f((m - m_new) * sl2);
+    l *= alpha;
+    m = m_new;
+  }
+  return rescale;
+}
+
+// P = 2^(S * sl2 - m * sl2) packed to bf16 into r[0, BK/2), fp32 partial row sums in acc.
+template <int BK>
+__device__ __forceinline__ void exp_tile(uint32_t* r, float sl2, float m, float2 (&acc)[2]) {
+  const float base = (m == -INFINITY) ? 0.f : m * sl2;
+  const float2 sc = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+  acc[0] = make_float2(0.f, 0.f);
+  acc[1] = make_float2(0.f, 0.f);
+  exp_pack_64<0>(r, sc, nb, acc);
+  if (BK == 128) exp_pack_64<64 % BK>(r, sc, nb, acc);
+}
+
+
 #endif  // __CUDACC__
 
 }  // namespace svg

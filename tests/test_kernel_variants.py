@@ -1,0 +1,48 @@
+"""The selectable two-SM kernels (SVG_KERNEL=pair: 512-row items, two halves per SM; SVG_KERNEL=pair1:
+one 128-row half per SM, key tiles alternating between two softmax groups) against the oracle.
+The kernel choice is read once per process, so each runs in a child process."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r"""
+import sys
+sys.path.insert(0, {root!r})
+from block_sparse_spatio_flash_b200 import synthetic as syn
+from tests import gpu_path as gp
+cases = [
+    (syn.Workload("medium_1200", frames=5, grid_h=12, grid_w=20, routes=(0, 1, 0, 1), d=128, frame_window=1,
+                  spatial_band=20), dict()),
+    (syn.Workload("medium_1200", frames=5, grid_h=12, grid_w=20, routes=(0, 1, 0, 1), d=128, frame_window=1,
+                  spatial_band=20), dict(bq=256, bk=64)),
+    (syn.Workload("rounded_1200", frames=5, grid_h=12, grid_w=20, routes=(1, 0), d=128, frame_window=1,
+                  spatial_band=20, variant=1), dict()),
+    (syn.Workload("sparse_rounded", frames=3, grid_h=16, grid_w=32, routes=(1,), d=128, frame_window=0,
+                  spatial_band=0, sink_frames=0, variant=1), dict()),
+]
+for w, kw in cases:
+    for mode in (0, 1):
+        q, k, v = syn.make_qkv(w, seed_offset=41)
+        out, lse, st = gp.run_path(w, q, k, v, mode=mode, **kw)
+        assert st == 0, st
+        gp.compare_rows(w, q, k, v, out, lse, variant=w.variant, **kw)
+    q, k, v = syn.make_qkv(w, seed_offset=43)
+    out, lse, st = gp.run_path(w, q, k, v, dense=True, bk=kw.get("bk", 128))
+    assert st == 0, st
+    gp.compare_rows(w, q, k, v, out, lse, all_kept=True)
+print("ok")
+"""
+
+
+@pytest.mark.parametrize("kernel", ["pair", "pair1"])
+def test_two_sm_kernels_match_oracle(kernel):
+    env = dict(os.environ, SVG_KERNEL=kernel)
+    r = subprocess.run([sys.executable, "-c", CHILD.format(root=ROOT)], env=env, cwd=ROOT, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), (r.stdout[-2000:], r.stderr[-4000:])
