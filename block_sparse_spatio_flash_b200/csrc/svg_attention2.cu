@@ -11,7 +11,7 @@
 //    rows and HALF of every K tile (BK/2 keys) and HALF of every V tile (64 of the 128 head
 //    dimensions), so each SM moves half the K/V bytes of the one-SM kernel from L2 into shared
 //    memory while receiving its full 128 x BK scores and 128 x 128 outputs in its own TMEM;
-//  * per CTA: warp 8 loads (TMA, no multicast) Q halves and its K/V halves; warps 0-3 / 4-7
+//  * per CTA: warp 8 loads (TMA, each CTA its own copy) Q halves and its K/V halves; warps 0-3 / 4-7
 //    are the softmax groups of the two halves; warp 9 of the even CTA issues the MMAs;
 //  * completion of every TMA copy of both CTAs is counted on the even CTA's barriers; MMA
 //    completion is signalled to the barriers of both CTAs (one commit per CTA); the odd CTA's

@@ -292,7 +292,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// 3-D tiled TMA load global -> shared, completion counted on `bar` (bytes). No multicast.
+// 3-D tiled TMA load global -> shared of this CTA, completion counted on `bar` (bytes).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                             int c2) {
   asm volatile(
@@ -455,7 +455,7 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t a, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 // TMA load into this CTA's shared memory whose completion is counted on an mbarrier of either
-// CTA of the pair (bar = shared::cluster address). No multicast.
+// CTA of the pair (bar = shared::cluster address); the data lands in the issuing CTA only.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
                                                  int c2) {
   asm volatile(
