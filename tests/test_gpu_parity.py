@@ -453,3 +453,26 @@ def test_fused_order_pages_mixed(S):
     got, _, st = gp.run_fused(w, q, k, v, lse=False)
     assert st == 0
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- limits
+def test_max_heads_small_geometry(S):
+    """4,096 heads (the ABI's limit) of a one-frame 8 x 8 geometry, alternating routes: the route bit
+    set, the work counter and the permutation at their largest head index; sampled heads checked."""
+    routes = tuple(h % 2 for h in range(4096))
+    w = syn.Workload("max_heads", frames=2, grid_h=4, grid_w=8, routes=routes, d=64, frame_window=0,
+                     spatial_band=3, bq=64, bk=64)
+    q, k, v = syn.make_qkv(w, seed_offset=51)
+    out, lse, st = gp.run_path(w, q, k, v)
+    assert st == 0
+    heads = [0, 1, 2047, 2048, 4094, 4095]
+    for h in heads:
+        rows = np.arange(w.tokens)
+        ref, _ = gp.oracle_rows(w, q, k, v, h, rows)
+        got = out[h].to(torch.float64).numpy()
+        assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= gp.REL_L2_TOL, h
+
+
+def test_smoke_entry_point(S):
+    import __graft_entry__
+    __graft_entry__.smoke()
