@@ -31,13 +31,19 @@
  *     device memory on any call.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). All device
  *     work is enqueued asynchronously on it; only svg_tilemap_summary and svg_read_status
- *     synchronise (that stream only).
+ *     synchronise (that stream only), and svg_attention_fwd_host, which works on host buffers
+ *     through streams of its own, returns when its result is on the host.
  *   - Host arrays (`h_route`) are read during the call and may be freed when it returns.
  *   - Return value: SVG_OK (0) or a negative SVG_ERR_* code; nothing is enqueued when an
  *     argument check fails. Errors detected on the device (a wait that timed out, a tile map
  *     built for other parameters) are written to the status word (see svg_read_status).
  *   - Requires a compute capability 10.0 device (B200, sm_100a); otherwise
  *     SVG_ERR_UNSUPPORTED.
+ *   - Environment (read by the host code): SVG_KERNEL=pair or SVG_KERNEL=pair1 (read once per
+ *     process) makes d = 128 attention run on the two-SM kernels instead of the one-SM kernel,
+ *     with the same results up to rounding; SVG_TEST_STALL=1 (read on every call) is a test hook
+ *     that makes an attention launch wait on a barrier nothing completes, so that it ends with
+ *     SVG_ERR_TIMEOUT in its status word after the wait limit (2 s).
  */
 #ifndef SVG_H_
 #define SVG_H_
@@ -182,7 +188,7 @@ int svg_dense_attention_fwd(const void *q, const void *k, const void *v, void *o
                             void *stream);
 
 /*
- * Allocation-free variant of svg_attention_fwd. The paper has no counterpart; it exists for
+ * Allocation-free variant of svg_attention_fwd. The case study has no counterpart; it exists for
  * callers that cannot allocate device memory themselves, e.g. a plugin inside a host
  * framework that hands it only the input and output buffers, or a server that forbids
  * device allocation after start-up because cudaMalloc may synchronise the device and
