@@ -434,7 +434,9 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
 
 def other_workloads(S, P, stream, dev):
     """Attention time (split mode, permuted inputs, 128 x 128 tiles) of the other workloads of the
-    pages' shapes: all-temporal and mixed heads at 75,600 tokens, mixed heads at 302,400 (1440p)."""
+    pages' shapes: all-temporal and mixed heads at 75,600 tokens, mixed heads at 302,400 (1440p);
+    next to it the fused-order call (svg_attention_fwd_fused on original-order tensors) and the
+    permuted path with its four permutation passes."""
     res = {}
     for w in (syn.TEMPORAL_75K, syn.MIXED_75K, syn.P1440):
         g = S.make_geom(w.frames, w.grid_h, w.grid_w)
@@ -445,7 +447,6 @@ def other_workloads(S, P, stream, dev):
         qp, kp, vp = (torch.empty_like(q) for _ in range(3))
         for a, b in ((q, qp), (k, kp), (v, vp)):
             S.svg_permute(a, b, routes, g, m)
-        del q, k, v
         o = torch.empty_like(qp)
         ws, summ = [None, None], {}
         for c in sorted(set(routes)):
@@ -455,12 +456,17 @@ def other_workloads(S, P, stream, dev):
         sc = S.alloc_scratch(dev)
         ms = time_events(lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, scratch=sc), 5,
                          stream)
+        # the same call with the permutation inside the kernel (original-order tensors)
+        ms_fused = time_events(
+            lambda: S.svg_attention_fwd_fused(q, k, v, o, routes, ws[0], ws[1], g, m, t, scratch=sc), 3, stream)
+        ms_perm = time_events(lambda: S.svg_permute(q, qp, routes, g, m), 3, stream)
         eff, vis, _ = workload_flops(w, summ)
         res[w.name] = {"ms": ms, "effective_tflops": eff / (ms * 1e-3) / 1e12,
                        "visited_tflops": vis / (ms * 1e-3) / 1e12,
                        "visited_frac_of_peak": vis / (ms * 1e-3) / 1e12 / float(P["bf16_tflops"]),
+                       "fused_order_ms": ms_fused, "permuted_path_ms": ms + 4 * ms_perm,
                        "status": S.svg_read_status(sc)}
-        del qp, kp, vp, o, ws
+        del q, k, v, qp, kp, vp, o, ws
         torch.cuda.empty_cache()
     return res
 
