@@ -427,9 +427,48 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
     out["route_ms"] = time_events(lambda: S.svg_route_heads(q, k, v, g, m, rows, rt, work=work), 5, stream)
     out["route_rows_per_head"] = int(rows.numel())
     out["workloads"] = other_workloads(S, P, stream, dev)
+    out["tile_sweep_mixed_75600"] = tile_sweep(S, stream, dev)
     st = S.svg_read_status(scratch)
     out["status"] = st
     return out
+
+
+def tile_sweep(S, stream, dev):
+    """mixed_75600 (5 spatial + 5 temporal heads) over query tiles {128, 256, 512} x key tiles
+    {64, 128}, exact and rounded masks: boundary-tile share of the visited tiles, visited share of
+    all tiles, kept-pair share, and the attention time."""
+    w = syn.MIXED_75K
+    routes = list(w.routes)
+    g = S.make_geom(w.frames, w.grid_h, w.grid_w)
+    q, k, v = (x.to(dev) for x in syn.make_qkv(w))
+    qp, kp, vp = (torch.empty_like(q) for _ in range(3))
+    m0 = S.make_mask(w.frame_window, w.spatial_band, w.sink_frames, S.SVG_MASK_EXACT, w.layout)
+    for a, b in ((q, qp), (k, kp), (v, vp)):
+        S.svg_permute(a, b, routes, g, m0)
+    del q, k, v
+    o = torch.empty_like(qp)
+    sc = S.alloc_scratch(dev)
+    res = {}
+    for bq, bk in syn.TILE_SWEEP:
+        t = S.make_tile(bq, bk)
+        for var, name in ((S.SVG_MASK_EXACT, "exact"), (S.SVG_MASK_ROUNDED, "rounded")):
+            m = S.make_mask(w.frame_window, w.spatial_band, w.sink_frames, var, w.layout)
+            ws, sm = [None, None], {}
+            for c in (0, 1):
+                ws[c] = S.alloc_workspace(g, t, dev)
+                S.svg_build_tilemap(g, m, t, c, ws[c])
+                sm[c] = S.svg_tilemap_summary(ws[c])
+            ms = time_events(lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, scratch=sc),
+                             3, stream)
+            vis = sum(sm[c].n_full + sm[c].n_boundary for c in (0, 1))
+            tot = sum(sm[c].n_full + sm[c].n_boundary + sm[c].n_empty for c in (0, 1))
+            kept = sum(sm[c].retained_map * routes.count(c) for c in (0, 1))
+            res[f"{bq}x{bk}-{name}"] = {"ms": ms, "boundary_frac_of_visited": sum(sm[c].n_boundary for c in (0, 1)) / vis,
+                                        "visited_frac_of_all": vis / tot,
+                                        "retained_frac": kept / (w.heads * w.tokens ** 2)}
+            del ws
+    res["status"] = S.svg_read_status(sc)
+    return res
 
 
 def other_workloads(S, P, stream, dev):
