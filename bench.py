@@ -473,11 +473,13 @@ def tile_sweep(S, stream, dev):
 
 def other_workloads(S, P, stream, dev):
     """Attention time (split mode, permuted inputs, 128 x 128 tiles) of the other workloads of the
-    pages' shapes: all-temporal and mixed heads at 75,600 tokens, mixed heads at 302,400 (1440p);
+    pages' shapes: all-temporal heads at 75,600 tokens (sink-prefix and fully space-major token
+    orders), mixed heads at 75,600 tokens, mixed heads at 302,400 (1440p);
     next to it the fused-order call (svg_attention_fwd_fused on original-order tensors) and the
     permuted path with its four permutation passes."""
     res = {}
-    for w in (syn.TEMPORAL_75K, syn.MIXED_75K, syn.P1440):
+    temporal_fsm = syn.TEMPORAL_75K.replace(name="temporal_75600_full_space_major", layout=syn.LAYOUT_FULL_SPACE_MAJOR)
+    for w in (syn.TEMPORAL_75K, temporal_fsm, syn.MIXED_75K, syn.P1440):
         g = S.make_geom(w.frames, w.grid_h, w.grid_w)
         m = S.make_mask(w.frame_window, w.spatial_band, w.sink_frames, w.variant, w.layout)
         t = S.make_tile(w.bq, w.bk)
