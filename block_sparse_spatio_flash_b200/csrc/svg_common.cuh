@@ -391,13 +391,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       SVG_W8(0), SVG_W8(8), SVG_W8(16), SVG_W8(24)
       : "memory");
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      SVG_W8(0), SVG_W8(8)
-      : "memory");
-}
 
 // Shared-memory matrix descriptor (tcgen05 format): start>>4 [0,14), LBO>>4 [16,30),
 // SBO>>4 [32,46), version 1 at bit 46, layout type [61,64) (2 = 128-byte swizzle).
@@ -506,7 +499,8 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
-// 2^x on the FMA / integer pipes, to take part of the exponentials off the MUFU unit.
+// 2^x on the FMA / integer pipes, to take part of the exponentials off the MUFU unit (used two
+// lanes at a time by exp2_poly2 below).
 // Cody-Waite style range reduction: n = round(x) (by the 1.5*2^23 rounding trick), f = x - n in
 // [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
 // error on [-1/2, 1/2] (fitted by linear programming, max rel. error 7.5e-5, far below the bf16
@@ -515,14 +509,6 @@ __device__ __forceinline__ float ex2f(float x) {
 // too small to move any finite sum; a row whose every score is masked is zeroed by its caller.
 constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f, kExpC2 = 2.426111251e-01f,
                 kExpC3 = 5.517166853e-02f;
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float r = xc + 12582912.f;  // 1.5 * 2^23: n sits in the low mantissa bits of r
-  const float n = r - 12582912.f;
-  const float f = xc - n;
-  const float p = fmaf(fmaf(fmaf(kExpC3, f, kExpC2), f, kExpC1), f, kExpC0);
-  return __uint_as_float((__float_as_uint(r) << 23) + __float_as_uint(p));
-}
 
 // Column pairs (mod 8) whose exponentials are computed by exp2_poly2 instead of ex2.approx.
 #ifndef SVG_POLY_MASK
@@ -536,7 +522,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Two-lane form of exp2_poly on the packed fp32x2 pipe: the rounding adds, the reduced argument
+// 2^x of two lanes on the packed fp32x2 pipe, by the method above: the rounding adds, the reduced argument
 // and the three polynomial steps are one FADD2 / FFMA2 each for both lanes; the clamp and the
 // exponent insertion (one integer multiply-add) stay per lane.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
