@@ -160,6 +160,13 @@ def oracle_sample(w, q, k, v, rows_per_head):
     return time.perf_counter() - t0, nrows, oracle.num_threads()
 
 
+def oracle_full_call_seconds(w, sec, nrows, fixed):
+    """Full-call oracle time from a row sample: the once-per-head part (widening K and V to fp64,
+    measured with one row per head) plus the per-row part of the sample scaled to every row."""
+    per_row = max(sec - fixed, 0.0) / nrows
+    return fixed + per_row * (w.tokens * w.heads)
+
+
 def closed_form_effective_flops(w):
     """4*d*retained for the exact masks, from the oracle's closed-form-pinned brute force is
     too slow here; the tile-map summary gives the same number on the GPU path. For the CPU
@@ -180,11 +187,12 @@ def run_reference(args, w, world, rank):
     rows = args.ref_rows
     for _ in range(args.warmup if args.warmup < 1 else 1):
         oracle_sample(w, q, k, v, max(4, rows // 8))
+    fixed, _, _ = oracle_sample(w, q, k, v, 1)  # the once-per-head part of a call
     times = []
     nthreads = 1
     for _ in range(args.steps):
         sec, nrows, nthreads = oracle_sample(w, q, k, v, rows)
-        times.append(sec * (w.tokens * w.heads) / nrows)  # extrapolated full-call seconds
+        times.append(oracle_full_call_seconds(w, sec, nrows, fixed))
     t = statistics.mean(times)
     value = eff / t / 1e12
     line = {
@@ -193,8 +201,9 @@ def run_reference(args, w, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
-                         "sample": f"{rows} seeded query rows per head x {w.heads} heads per step; full-call time "
-                                   f"extrapolated linearly by rows"},
+                         "sample": f"{rows} seeded query rows per head x {w.heads} heads per step; full-call time = "
+                                   f"once-per-head part ({fixed:.2f} s, timed with one row per head) + per-row "
+                                   f"part scaled to all rows"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -217,7 +226,7 @@ def main():
                     help="only the timed steps (no side measurements, e2e or CPU baseline): for profiler runs")
     ap.add_argument("--heads", type=int, default=0, help="use only the first H heads of the workload")
     ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
-    ap.add_argument("--ref-rows", type=int, default=48, help="oracle rows per head per --impl reference step")
+    ap.add_argument("--ref-rows", type=int, default=96, help="oracle rows per head per --impl reference step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -315,11 +324,13 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.quick:
+        fixed, _, _ = oracle_sample(w, q_cpu, k_cpu, v_cpu, 1)
         sec, nrows, nthreads = oracle_sample(w, q_cpu, k_cpu, v_cpu, args.cpu_rows)
-        full = sec * (w.tokens * w.heads) / nrows
+        full = oracle_full_call_seconds(w, sec, nrows, fixed)
         cpu = {"value": eff_flop / full / 1e12, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
                "sample": f"{args.cpu_rows} seeded query rows per head x {w.heads} heads ({nrows} rows, "
-                         f"{sec:.1f} s); full-call time extrapolated linearly by rows = {full:.1f} s",
+                         f"{sec:.1f} s); full-call time = once-per-head part ({fixed:.2f} s, one row per head) "
+                         f"+ per-row part scaled to all rows = {full:.1f} s",
                "ms_per_call_extrapolated": full * 1e3}
 
     if world > 1:
