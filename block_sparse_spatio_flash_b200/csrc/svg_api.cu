@@ -21,7 +21,7 @@ int launch_attention_pair1(const AttnParams& P, int bk, cudaStream_t st);
 size_t route_work_bytes(int heads, int64_t N, int d, int n_rows);
 int launch_route(const void* q, const void* k, const void* v, int heads, int N, int d, float scale, svg_geom geom,
                  svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
-                 cudaStream_t st);
+                 int num_sms, cudaStream_t st);
 }  // namespace svg
 
 using namespace svg;
@@ -467,11 +467,12 @@ int svg_route_heads(const void* q, const void* k, const void* v, int32_t heads, 
   if ((int64_t)geom.frames * geom.grid_h * geom.grid_w != tokens) return SVG_ERR_ARG;
   if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
   if (work_bytes < svg_route_work_bytes(heads, tokens, d, n_rows)) return SVG_ERR_WORKSPACE;
-  int rc = device_info(nullptr);
+  int num_sms = 0;
+  int rc = device_info(&num_sms);
   if (rc) return rc;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   return launch_route(q, k, v, heads, (int)tokens, d, sc, geom, mask, d_rows, n_rows, d_work, d_route, d_err,
-                      static_cast<cudaStream_t>(stream));
+                      num_sms, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------------------

@@ -32,11 +32,29 @@ __host__ __device__ inline int route_chunks(int64_t N) {
   const int64_t c = (N + kRouteChunkKeys - 1) / kRouteChunkKeys;
   return (int)(c < 1 ? 1 : (c > kRouteMaxChunks ? kRouteMaxChunks : c));
 }
-// Keys per chunk (a multiple of the tile) and the number of non-empty chunks.
-inline int route_chunk_len(int64_t N) {
-  const int G = route_chunks(N);
+// Keys per chunk (a multiple of the tile) when the keys are cut into G chunks.
+inline int route_chunk_len(int64_t N, int G) {
   const int64_t per = (N + G - 1) / G;
   return (int)((per + kRouteKeys - 1) / kRouteKeys * kRouteKeys);
+}
+// Chunks for this launch: the count (at most route_chunks(N), the count the work buffer is sized
+// for) whose blocks fill the GPU's 2 x SM block slots best over whole waves -- a last, mostly empty
+// wave costs as much as a full one; among equals the larger count (shorter blocks).
+inline int route_launch_chunks(int64_t N, int row_blocks, int heads, int num_sms) {
+  const int64_t per_chunk = (int64_t)row_blocks * heads;
+  const int64_t slots = 2 * (int64_t)(num_sms > 0 ? num_sms : 1);
+  int best = 1;
+  double best_fill = -1.0;
+  for (int g = 1; g <= route_chunks(N); ++g) {
+    const int64_t blocks = per_chunk * g;
+    const int64_t waves = (blocks + slots - 1) / slots;
+    const double fill = (double)blocks / (double)(waves * slots);
+    if (fill >= best_fill - 1e-9) {
+      best_fill = fill;
+      best = g;
+    }
+  }
+  return best;
 }
 
 size_t route_rowerr_bytes(int heads, int n_rows) {
@@ -330,7 +348,7 @@ static cudaError_t launch_partial(const RouteParams& P, int nblk_rows, int nchun
 
 int launch_route(const void* q, const void* k, const void* v, int heads, int N, int d, float scale, svg_geom geom,
                  svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
-                 cudaStream_t st) {
+                 int num_sms, cudaStream_t st) {
   RouteParams P;
   P.q = static_cast<const __nv_bfloat16*>(q);
   P.k = static_cast<const __nv_bfloat16*>(k);
@@ -343,13 +361,13 @@ int launch_route(const void* q, const void* k, const void* v, int heads, int N, 
   P.gt = make_geom(geom, mask, SVG_ROUTE_TEMPORAL);
   P.rows = rows;
   P.n_rows = n_rows;
-  P.chunk = route_chunk_len(N);
+  const int nblk_rows = (n_rows + kRouteRows - 1) / kRouteRows;
+  P.chunk = route_chunk_len(N, route_launch_chunks(N, nblk_rows, heads, num_sms));
   P.G = (N + P.chunk - 1) / P.chunk;  // non-empty chunks, at most route_chunks(N)
   P.rowerr = static_cast<float*>(work);
   P.part = reinterpret_cast<float*>(static_cast<unsigned char*>(work) + route_rowerr_bytes(heads, n_rows));
   P.route = route;
   P.err = err;
-  const int nblk_rows = (n_rows + kRouteRows - 1) / kRouteRows;
   cudaError_t e = d == 128 ? launch_partial<128>(P, nblk_rows, P.G, st) : launch_partial<64>(P, nblk_rows, P.G, st);
   if (e != cudaSuccess) return record_cuda_error("launch route_partial_kernel", e);
   route_merge_kernel<<<dim3(n_rows, heads), 32, 0, st>>>(P);
