@@ -411,6 +411,13 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
                                                        mode=S.SVG_MODE_SPLIT, scratch=scratch), 5, stream)
     out["split_ms"] = ms_split
     out["split_vs_dense"] = out["dense_ms"] / ms_split
+    # QK^T on the 8-bit path (e4m3 copies of the permuted Q and K): an opt-in variant, not the headline
+    q8, k8 = qp.to(torch.float8_e4m3fn), kp.to(torch.float8_e4m3fn)
+    ms = time_events(lambda: S.svg_attention_fwd_qk8(q8, k8, vp, o, routes, ws[0], ws[1], g, m, t, scratch=scratch),
+                     5, stream)
+    out["qk8_ms"] = ms
+    out["qk8_vs_split"] = ms_split / ms
+    del q8, k8
     # rounded (tile-aligned) masks
     mr = S.make_mask(w.frame_window, w.spatial_band, w.sink_frames, S.SVG_MASK_ROUNDED, w.layout)
     wr = [None, None]

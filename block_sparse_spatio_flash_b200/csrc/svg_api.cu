@@ -114,6 +114,25 @@ int encode_qkv_map(CUtensorMap* m, const void* base, int heads, int tokens, int 
   return SVG_OK;
 }
 
+// [heads, tokens, d] e4m3 (one byte per element, d = 128): box 128 columns (one 128-byte swizzle
+// row) x box_rows rows.
+int encode_qk8_map(CUtensorMap* m, const void* base, int heads, int tokens, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return record_cuda_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", (int)cudaErrorSymbolNotFound);
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)tokens, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)tokens * d};
+  cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (e4m3): CUresult %d", (int)r);
+    return SVG_ERR_CUDA;
+  }
+  return SVG_OK;
+}
+
 // [heads * tokens, d] bf16 viewed as rows, box 64 columns x 1 row, 128-byte swizzle: the map
 // for 4-row gathers of arbitrary rows.
 int encode_rows_map(CUtensorMap* m, const void* base, int heads, int64_t tokens, int d) {
@@ -166,12 +185,14 @@ int check_qkvo(const void* q, const void* k, const void* v, const void* o, const
 int run_attention(const void* q, const void* k, const void* v, void* o, float* lse, int heads, int64_t tokens,
                   int d, float scale, const uint8_t* h_route, const void* ws_sp, const void* ws_tm,
                   const svg_geom* geom, const svg_mask* mask, int bq, int bk, int mode, bool dense,
-                  void* scratch, size_t scratch_bytes, int32_t* d_status, cudaStream_t st, bool fused = false) {
+                  void* scratch, size_t scratch_bytes, int32_t* d_status, cudaStream_t st, bool fused = false,
+                  bool qk8 = false) {
   int rc = check_qkvo(q, k, v, o, lse, heads, tokens, d);
   if (rc) return rc;
   if (!scratch || scratch_bytes < kScratchBytes || !aligned(scratch, 16)) return SVG_ERR_ARG;
   if (d_status && !aligned(d_status, 4)) return SVG_ERR_ARG;
   if (bk != 64 && bk != 128) return SVG_ERR_UNSUPPORTED;
+  if (qk8 && (d != 128 || fused)) return SVG_ERR_UNSUPPORTED;  // e4m3 QK^T: d = 128, permuted order
   int num_sms = 0;
   rc = device_info(&num_sms);
   if (rc) return rc;
@@ -181,8 +202,8 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   std::lock_guard<std::mutex> lock(mu);
   memset(&P, 0, sizeof(P));
   const int N = (int)tokens;
-  const bool pair = use_pair_kernel(d) && !fused;
-  const bool pair1 = use_pair1_kernel(d) && !fused && !pair;
+  const bool pair = use_pair_kernel(d) && !fused && !qk8;
+  const bool pair1 = use_pair1_kernel(d) && !fused && !pair && !qk8;
   P.H = heads;
   P.N = N;
   P.nk = (N + bk - 1) / bk;
@@ -197,6 +218,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   P.bkm = bk;
   P.naive = mode == SVG_MODE_NAIVE ? 1 : 0;
   P.fused = fused && !dense ? 1 : 0;
+  P.qk8 = qk8 ? 1 : 0;
   {  // test hook, read on every call: SVG_TEST_STALL=1 makes the launch time out on purpose
     const char* ts = getenv("SVG_TEST_STALL");
     P.inject_stall = (ts && ts[0] == '1' && !pair && !pair1) ? 1 : 0;
@@ -250,8 +272,13 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   }
   // TMA boxes: Q 128 rows; one-SM kernel K and V bk rows; SM-pair kernel: each SM loads bk/2
   // keys of K (all 128 dims) and all bk keys of V for 64 of the dims.
-  if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
-  if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, (pair || pair1) ? bk / 2 : bk))) return rc;
+  if (qk8) {
+    if ((rc = encode_qk8_map(&P.tm_q, q, heads, N, d, 128))) return rc;
+    if ((rc = encode_qk8_map(&P.tm_k, k, heads, N, d, bk))) return rc;
+  } else {
+    if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
+    if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, (pair || pair1) ? bk / 2 : bk))) return rc;
+  }
   if ((rc = encode_qkv_map(&P.tm_v, v, heads, N, d, bk))) return rc;
   if (P.fused && P.uses[SVG_ROUTE_TEMPORAL]) {
     if ((rc = encode_rows_map(&P.tm_q2, q, heads, N, d))) return rc;
@@ -428,6 +455,15 @@ int svg_attention_fwd_fused(const void* q, const void* k, const void* v, void* o
   return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
                        tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
                        static_cast<cudaStream_t>(stream), true);
+}
+
+int svg_attention_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, float* lse, int32_t heads,
+                          int64_t tokens, int32_t d, float scale, const uint8_t* h_route, const void* d_ws_spatial,
+                          const void* d_ws_temporal, svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
+                          void* d_scratch, size_t scratch_bytes, int32_t* d_status, void* stream) {
+  return run_attention(q8, k8, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
+                       tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
+                       static_cast<cudaStream_t>(stream), false, true);
 }
 
 int svg_dense_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,

@@ -33,12 +33,18 @@ constexpr int kMmaWarp = 9;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 
-template <int D, int BK>
+// QK8: Q and K in e4m3 (one byte per element, d = 128: one 128-byte swizzle chunk per row), QK^T on
+// the tensor core's 8-bit path; V, P and O as in the bf16 path.
+template <int D, int BK, bool QK8 = false>
 struct Cfg {
-  static constexpr int kChunks = D / 64;            // 128-byte swizzle chunks per row
-  static constexpr int kQHalfBytes = 128 * D * 2;
+  static constexpr int kChunks = D / 64;            // 128-byte swizzle chunks per bf16 row (V)
+  static constexpr int kQKChunks = QK8 ? D / 128 : D / 64;  // the same for a Q or K row
+  static constexpr int kQKColsPerChunk = QK8 ? 128 : 64;
+  static constexpr int kQHalfBytes = 128 * D * (QK8 ? 1 : 2);
   static constexpr int kQBytes = 2 * kQHalfBytes;
-  static constexpr int kTileBytes = BK * D * 2;     // one K or one V tile
+  static constexpr int kKBytes = BK * D * (QK8 ? 1 : 2);
+  static constexpr int kVBytes = BK * D * 2;
+  static constexpr int kTileBytes = BK * D * 2;     // ring slot: one K or one V tile
   static constexpr int kStages = (160 * 1024) / kTileBytes;
   static constexpr int kDataBytes = kQBytes + kStages * kTileBytes;
   static constexpr int kSmemBytes = kDataBytes + 1024 /*control*/ + 1024 /*alignment slack*/;
@@ -177,9 +183,9 @@ __device__ ItemInfo decode_item(const AttnParams& P, uint32_t idx) {
 }
 
 // ---------------------------------------------------------------------------------------
-template <int D, int BK>
+template <int D, int BK, bool QK8 = false>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
-  using C = Cfg<D, BK>;
+  using C = Cfg<D, BK, QK8>;
   constexpr int NS = C::kStages;
   using K = Ctl<NS>;
   static_assert(K::kBytes <= 1024, "control block");
@@ -288,8 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
               tma_gather4(sQ + h * C::kQHalfBytes + ch * (128 * 128) + lane * 512, &P.tm_q2, c.q_full(), ch * 64, rr[0],
                           rr[1], rr[2], rr[3]);
           } else if (lane == 0) {
-            for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_3d(sQ + h * C::kQHalfBytes + ch * (128 * 128), &P.tm_q, c.q_full(), ch * 64, p0, inf.head);
+            for (int ch = 0; ch < C::kQKChunks; ++ch)
+              tma_load_3d(sQ + h * C::kQHalfBytes + ch * (128 * 128), &P.tm_q, c.q_full(), ch * C::kQKColsPerChunk, p0,
+                          inf.head);
           }
         }
         q_issued = true;
@@ -310,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             ok = false;
             break;
           }
-          if (lane == 0) mbar_expect_tx(c.kv_full(st), C::kTileBytes);
+          if (lane == 0) mbar_expect_tx(c.kv_full(st), w == 0 ? C::kKBytes : C::kVBytes);
           __syncwarp();
           const uint32_t dst = sRing + st * C::kTileBytes;
           if (gat) {
@@ -319,8 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 tma_gather4(dst + ch * (BK * 128) + lane * 512, w == 0 ? &P.tm_k2 : &P.tm_v2, c.kv_full(st), ch * 64,
                             rr[0], rr[1], rr[2], rr[3]);
           } else if (lane == 0) {
-            for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_3d(dst + ch * (BK * 128), w == 0 ? &P.tm_k : &P.tm_v, c.kv_full(st), ch * 64, row0, inf.head);
+            if (w == 0) {
+              for (int ch = 0; ch < C::kQKChunks; ++ch)
+                tma_load_3d(dst + ch * (BK * 128), &P.tm_k, c.kv_full(st), ch * C::kQKColsPerChunk, row0, inf.head);
+            } else {
+              for (int ch = 0; ch < C::kChunks; ++ch)
+                tma_load_3d(dst + ch * (BK * 128), &P.tm_v, c.kv_full(st), ch * 64, row0, inf.head);
+            }
           }
           ++kv_pos;
         }
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   } else if (!skip_all && warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(BK, false);
+      constexpr uint32_t idesc_s = QK8 ? idesc_e4m3_f32(BK) : idesc_bf16_f32(BK, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(D, true);
       // Descriptors are built once; per k-step and per ring slot only the start-address
       // field (bits [0,14), address >> 4) moves, and no address exceeds 256 KB, so a plain add
@@ -402,12 +414,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 k_ready = true;
               }
               const uint64_t qd = qdesc + ((h * C::kQHalfBytes) >> 4);
+              if constexpr (QK8) {
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                // 16 bf16 = 32 bytes along K inside a 128-byte swizzle atom; 64 columns per atom
-                const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
-                const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
-                umma_ss(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < D / 32; ++kk) {
+                  // 32 e4m3 = 32 bytes along K inside a 128-byte swizzle atom; 128 columns per atom
+                  const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                  const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
+                  umma_ss_f8(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
+                }
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  // 16 bf16 = 32 bytes along K inside a 128-byte swizzle atom; 64 columns per atom
+                  const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                  const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
+                  umma_ss(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
+                }
               }
               umma_commit(c.s_full(h));
             }
@@ -559,10 +581,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------------------------------
-template <int D, int BK>
+template <int D, int BK, bool QK8 = false>
 static int launch_t(const AttnParams& P, int grid, cudaStream_t st) {
-  using C = Cfg<D, BK>;
-  auto kern = attn_kernel<D, BK>;
+  using C = Cfg<D, BK, QK8>;
+  auto kern = attn_kernel<D, BK, QK8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return record_cuda_error("cudaFuncSetAttribute(attn_kernel)", e);
   kern<<<grid, kThreads, C::kSmemBytes, st>>>(P);
@@ -571,6 +593,11 @@ static int launch_t(const AttnParams& P, int grid, cudaStream_t st) {
 }
 
 int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st) {
+  if (P.qk8) {  // e4m3 Q and K: d = 128
+    if (d == 128 && bk == 128) return launch_t<128, 128, true>(P, grid, st);
+    if (d == 128 && bk == 64) return launch_t<128, 64, true>(P, grid, st);
+    return SVG_ERR_UNSUPPORTED;
+  }
   if (d == 128 && bk == 128) return launch_t<128, 128>(P, grid, st);
   if (d == 128 && bk == 64) return launch_t<128, 64>(P, grid, st);
   if (d == 64 && bk == 128) return launch_t<64, 128>(P, grid, st);

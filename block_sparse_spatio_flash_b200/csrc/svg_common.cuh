@@ -211,6 +211,8 @@ struct AttnParams {
   // and write O rows back to their original index.
   CUtensorMap tm_q2, tm_k2, tm_v2;
   int fused;
+  // QK^T operands in e4m3 (one byte per element): tm_q / tm_k then describe 1-byte tensors
+  int qk8;
   // Test hook: the softmax warps first wait on a barrier that nothing completes, so that the
   // bounded-wait / abort / drain path runs and the launch ends with SVG_ERR_TIMEOUT.
   int inject_stall;
@@ -344,6 +346,16 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, both e4m3 (kind::f8f6f4, K = 32 per instruction)
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // D[tmem] (+)= A[tmem] * B[smem]
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate) {
@@ -410,6 +422,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int n, bool b_mn_major, in
          | (1u << 7)                    // A format bf16
          | (1u << 10)                   // B format bf16
          | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(n >> 3) << 17)   // N / 8
+         | ((uint32_t)(m >> 4) << 24);  // M / 16
+}
+
+// Instruction descriptor, kind::f8f6f4: D fp32, A and B e4m3 (format code 0), both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n, int m = 128) {
+  return (1u << 4)                      // D format fp32
          | ((uint32_t)(n >> 3) << 17)   // N / 8
          | ((uint32_t)(m >> 4) << 24);  // M / 16
 }

@@ -83,6 +83,8 @@ _sig = {
                                                  _vp, _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _vp]),
     "svg_attention_fwd_fused": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp,
                                                _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
+    "svg_attention_fwd_qk8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp,
+                                             _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
     "svg_attention_host_buffer_bytes": (_sz, [_i64, _i32, _i32]),
     "svg_attention_fwd_host": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp, _vp,
                                               svg_geom, svg_mask, svg_tile, _i32, _i32, _vp, _sz]),
@@ -203,6 +205,17 @@ def svg_attention_fwd_fused(q, k, v, o, routes, ws_spatial, ws_temporal, geom, m
                                         _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile, mode,
                                         _ptr(scratch), scratch.numel() * scratch.element_size(), _ptr(status),
                                         _stream(stream)), "svg_attention_fwd_fused")
+    return o
+
+
+def svg_attention_fwd_qk8(q8, k8, v, o, routes, ws_spatial, ws_temporal, geom, mask, tile, mode=SVG_MODE_SPLIT,
+                          scratch=None, lse=None, scale: float = 0.0, status=None, stream=None) -> torch.Tensor:
+    """svg_attention_fwd with e4m3 Q and K (torch.float8_e4m3fn or uint8 [H, N, 128]); v / o bf16."""
+    heads, tokens, d = v.shape
+    _check(_lib.svg_attention_fwd_qk8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(o), _ptr(lse), heads, tokens, d, scale,
+                                      _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile, mode,
+                                      _ptr(scratch), scratch.numel() * scratch.element_size(), _ptr(status),
+                                      _stream(stream)), "svg_attention_fwd_qk8")
     return o
 
 

@@ -180,6 +180,22 @@ int svg_attention_fwd(const void *q, const void *k, const void *v, void *o, floa
                       svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
                       void *d_scratch, size_t scratch_bytes, int32_t *d_status, void *stream);
 
+/*
+ * svg_attention_fwd with QK^T on the tensor core's 8-bit path: q8 and k8 are e4m3 (one byte per
+ * element, [heads, tokens, d], d = 128, each head's rows in its token order -- svg_permute moves
+ * e4m3 rows when called with d = 64, since a 128-byte row is 64 bf16-sized elements); v, o, lse and
+ * every other argument as in svg_attention_fwd. `scale` multiplies the e4m3 dot products, so it
+ * carries any quantisation scales of Q and K (<= 0: 1/sqrt(d)). The scores are the exact fp32 sums of
+ * the e4m3 products; softmax, P (bf16) and P V are those of svg_attention_fwd, so the result is the
+ * attention of the dequantised Q and K. Not a counterpart of anything on the pages: an opt-in
+ * variant that halves the QK^T work and its shared-memory traffic. SVG_ERR_UNSUPPORTED for d != 128.
+ */
+int svg_attention_fwd_qk8(const void *q8, const void *k8, const void *v, void *o, float *lse,
+                          int32_t heads, int64_t tokens, int32_t d, float scale,
+                          const uint8_t *h_route, const void *d_ws_spatial, const void *d_ws_temporal,
+                          svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
+                          void *d_scratch, size_t scratch_bytes, int32_t *d_status, void *stream);
+
 /* Dense attention forward (every pair kept) with the same kernel and scheduler; the
  * in-repo baseline. Arguments as in svg_attention_fwd; bk in {64, 128}. */
 int svg_dense_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,

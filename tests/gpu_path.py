@@ -167,3 +167,31 @@ def lse_to_original(w: syn.Workload, lse):
         pi = oracle.perm_table(w.routes[h], w.layout, w.frames, w.frame_size, w.sink_frames)
         out[h] = lse[h, torch.as_tensor(pi)]
     return out
+
+
+def quantize_e4m3(x):
+    """bf16 -> e4m3 (round to nearest) -> bf16: the values the 8-bit QK^T path sees, exactly."""
+    return x.to(torch.float8_e4m3fn).to(torch.bfloat16)
+
+
+def run_qk8(w: syn.Workload, q, k, v, *, mode=0, variant=None, bq=None, bk=None):
+    """svg_attention_fwd_qk8 on e4m3 copies of q and k (q and k must already hold e4m3 values in bf16,
+    see quantize_e4m3). Returns (O [H, N, d] bf16 CPU in original order, status)."""
+    S = svg()
+    dev = torch.device("cuda")
+    g, m, t = geom_mask_tile(w, variant, bq, bk)
+    routes = list(w.routes)
+    qd, kd, vd = (x.to(dev).contiguous() for x in (q, k, v))
+    qp, kp, vp = (torch.empty_like(x) for x in (qd, kd, vd))
+    for src, dst in ((qd, qp), (kd, kp), (vd, vp)):
+        S.svg_permute(src, dst, routes, g, m, inverse=False)
+    q8, k8 = (x.to(torch.float8_e4m3fn).contiguous() for x in (qp, kp))  # exact: the values are e4m3
+    o = torch.empty_like(vp)
+    scratch = S.alloc_scratch()
+    maps = build_maps(w, g, m, t, routes)
+    S.svg_attention_fwd_qk8(q8, k8, vp, o, routes, maps[0], maps[1], g, m, t, mode=mode, scratch=scratch)
+    status = S.svg_read_status(scratch)
+    out = torch.empty_like(o)
+    S.svg_permute(o, out, routes, g, m, inverse=True)
+    torch.cuda.synchronize()
+    return out.cpu(), status

@@ -172,3 +172,14 @@ def test_host_entry_argument_checks(svg):
     assert f(h, h, h, h, 2, 512, 64, 0.0, routes, dbuf, dbuf, g, m, t, 0, 2, dbuf, need - 1) == -5  # buffer
     bad = (ctypes.c_uint8 * 2)(0, 3)
     assert f(h, h, h, h, 2, 512, 64, 0.0, bad, dbuf, dbuf, g, m, t, 0, 2, dbuf, need) == -1         # route
+
+
+def test_qk8_argument_checks(svg):
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    f = lib.svg_attention_fwd_qk8
+    f.argtypes = svg._sig["svg_attention_fwd_qk8"][1]
+    g, m, t = svg.make_geom(4, 8, 16), svg.make_mask(1, 16), svg.make_tile(64, 64)
+    routes = (ctypes.c_uint8 * 2)(0, 1)
+    p = ctypes.c_void_p(1 << 20)
+    assert f(p, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -2   # d = 64
+    assert f(None, p, p, p, None, 2, 512, 128, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -1  # null q8

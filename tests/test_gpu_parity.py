@@ -476,3 +476,38 @@ def test_max_heads_small_geometry(S):
 def test_smoke_entry_point(S):
     import __graft_entry__
     __graft_entry__.smoke()
+
+
+# ----------------------------------------------------------------------------- e4m3 QK^T
+@pytest.mark.parametrize("bq,bk", [(128, 128), (256, 64)])
+@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_qk8_matches_oracle_on_quantised_inputs(S, bq, bk, variant, mode):
+    """QK^T on the 8-bit path: the oracle sees the same e4m3 values (exact in bf16), so parity holds
+    with the bf16 path's tolerance."""
+    w = MEDIUM.replace(bq=bq, bk=bk, variant=variant)
+    q, k, v = syn.make_qkv(w, seed_offset=61)
+    q, k = gp.quantize_e4m3(q), gp.quantize_e4m3(k)
+    out, st = gp.run_qk8(w, q, k, v, mode=mode)
+    assert st == 0
+    gp.compare_rows(w, q, k, v, out, None, variant=variant, bq=bq, bk=bk)
+
+
+def test_qk8_pages_temporal_and_growing_maxima(S):
+    w = syn.TEMPORAL_75K.replace(sample_rows=256)
+    q, k, v = syn.make_qkv(w)
+    q, k = gp.quantize_e4m3(q), gp.quantize_e4m3(k)
+    out, st = gp.run_qk8(w, q, k, v)
+    assert st == 0
+    gp.compare_rows(w, q, k, v, out, None)
+    wm = MEDIUM
+    q, k, v = syn.make_qkv(wm, seed_offset=13)
+    k = k.float()
+    g = torch.Generator().manual_seed(77)
+    for h in range(wm.heads):
+        idx = torch.randperm(wm.tokens, generator=g)[:24]
+        k[h, idx] *= torch.linspace(2.0, 9.0, 24)[:, None]
+    q, k = gp.quantize_e4m3(q), gp.quantize_e4m3(k.to(torch.bfloat16))
+    out, st = gp.run_qk8(wm, q, k, v)
+    assert st == 0
+    gp.compare_rows(wm, q, k, v, out, None)
