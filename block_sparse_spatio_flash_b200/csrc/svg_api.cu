@@ -15,7 +15,7 @@ namespace svg {
 int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* ws, cudaStream_t st);
 int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const uint8_t* h_route, svg_geom geom,
                    svg_mask mask, int inverse, int num_sms, cudaStream_t st);
-int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st);
+int launch_attention(const AttnParams& P, int d, int bk, int grid, bool p_smem, cudaStream_t st);
 int launch_attention_pair(const AttnParams& P, int bk, int max_clusters, cudaStream_t st);
 int launch_attention_pair1(const AttnParams& P, int bk, cudaStream_t st);
 size_t route_work_bytes(int heads, int64_t N, int d, int n_rows);
@@ -172,6 +172,16 @@ bool use_pair1_kernel(int d) {
   return d == 128 && pair1;
 }
 
+// SVG_KERNEL=ps: the single-SM kernel with P staged in shared memory, so that the next key tile's
+// S is computed while the softmax of this one runs.
+bool use_p_smem() {
+  static const bool ps = [] {
+    const char* v = getenv("SVG_KERNEL");
+    return v && strcmp(v, "ps") == 0;
+  }();
+  return ps;
+}
+
 int check_qkvo(const void* q, const void* k, const void* v, const void* o, const float* lse, int heads,
                int64_t tokens, int d) {
   if (!q || !k || !v || !o) return SVG_ERR_ARG;
@@ -291,7 +301,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   if (pair) return launch_attention_pair(P, bk, (int)(P.n_items < num_sms / 2 ? P.n_items : num_sms / 2), st);
   if (pair1) return launch_attention_pair1(P, bk, st);
   const int grid = (int)(P.n_items < num_sms ? P.n_items : num_sms);
-  return launch_attention(P, d, bk, grid, st);
+  return launch_attention(P, d, bk, grid, use_p_smem(), st);
 }
 
 }  // namespace

@@ -16,6 +16,8 @@
 //  * warps 0-3 and 4-7 are two softmax groups, one per 128-row half, one thread per query
 //    row (= TMEM lane). While one group turns its S into P, the tensor core computes the
 //    other half's S and P V, so MMA and exponentials overlap;
+//  * option PS: P goes to shared memory instead, so the next tile's S is computed while the
+//    softmax of this tile runs (measured slower on B200; kept selectable);
 //  * O is rescaled (in TMEM) only when a row maximum grows by more than 2^8, which keeps
 //    the result exact while making the correction rare;
 //  * every wait is bounded by a wall-clock limit; a timeout sets the status word and all
@@ -35,25 +37,30 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 // QK8: Q and K in e4m3 (one byte per element, d = 128: one 128-byte swizzle chunk per row), QK^T on
 // the tensor core's 8-bit path; V, P and O as in the bf16 path.
-template <int D, int BK, bool QK8 = false>
+// PS: P goes to shared memory (same 128-byte swizzle layout as a Q half) instead of TMEM, and P V
+// reads it from there. S_h's TMEM columns are then free as soon as the softmax has loaded them,
+// so the next tile's S_h is computed while the softmax of this tile runs.
+template <int D, int BK, bool QK8 = false, bool PS = false>
 struct Cfg {
   static constexpr int kChunks = D / 64;            // 128-byte swizzle chunks per bf16 row (V)
   static constexpr int kQKChunks = QK8 ? D / 128 : D / 64;  // the same for a Q or K row
   static constexpr int kQKColsPerChunk = QK8 ? 128 : 64;
   static constexpr int kQHalfBytes = 128 * D * (QK8 ? 1 : 2);
   static constexpr int kQBytes = 2 * kQHalfBytes;
+  static constexpr int kPHalfBytes = PS ? 128 * BK * 2 : 0;
+  static constexpr int kPBytes = 2 * kPHalfBytes;
   static constexpr int kKBytes = BK * D * (QK8 ? 1 : 2);
   static constexpr int kVBytes = BK * D * 2;
   static constexpr int kTileBytes = BK * D * 2;     // ring slot: one K or one V tile
-  static constexpr int kStages = (160 * 1024) / kTileBytes;
-  static constexpr int kDataBytes = kQBytes + kStages * kTileBytes;
+  static constexpr int kStages = PS ? (224 * 1024 - kQBytes - kPBytes) / kTileBytes : (160 * 1024) / kTileBytes;
+  static constexpr int kDataBytes = kQBytes + kPBytes + kStages * kTileBytes;
   static constexpr int kSmemBytes = kDataBytes + 1024 /*control*/ + 1024 /*alignment slack*/;
   // TMEM columns: S (and P) of half h at 128*h, P (bf16 pairs) aliases the upper half of
   // S, O accumulators of half h at 256 + D*h.
   __host__ __device__ static constexpr uint32_t s_col(int h) { return 128u * h; }
   static constexpr uint32_t kPCol = BK / 2;
   __host__ __device__ static constexpr uint32_t o_col(int h) { return 256u + (uint32_t)D * h; }
-  static_assert(kStages >= 2, "ring too small");
+  static_assert(kStages >= (PS ? 3 : 2), "ring too small");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -69,13 +76,14 @@ struct ItemInfo {
 //   2NS + 0 / 1    q_full / q_free
 //   2NS + 2 + h    s_full[h]     S_h = Q_h K^T (and every earlier MMA) complete
 //   2NS + 4 + h    p_ready[h]    P_h in TMEM, O_h corrected (128 arrivals)
-//   2NS + 6 + h    o_done[h]     last P V of half h complete
+//   2NS + 6 + h    o_done[h]     last P V of half h complete (PS: every P V of half h, pv_done)
 //   2NS + 8 + h    o_free[h]     epilogue finished reading O_h (128 arrivals)
 //   2NS + 10 + i   item_full[i]  work item published in slot i
 //   2NS + 12 + i   item_empty[i] slot i read by the MMA warp and the 8 softmax warps
 //   2NS + 14       drain         final MMA completion
 //   2NS + 15       never         completed by nothing (test hook: a wait that runs out)
-//   2NS + 16 ...   two ItemInfo slots, TMEM base, abort flag, workspace check
+//   2NS + 16 + h   s_free[h]     (PS) S_h loaded by the softmax, its TMEM columns free (128 arrivals)
+//   2NS + 18 ...   two ItemInfo slots, TMEM base, abort flag, workspace check
 template <int NS>
 struct Ctl {
   uint32_t base;  // shared address of the control block
@@ -92,7 +100,8 @@ struct Ctl {
   __device__ __forceinline__ uint32_t item_empty(uint32_t i) const { return base + 8u * (2 * NS + 12 + i); }
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * (2 * NS + 14); }
   __device__ __forceinline__ uint32_t never() const { return base + 8u * (2 * NS + 15); }
-  static constexpr uint32_t kItemsOff = 8u * (2 * NS + 16);  // 2 x 40 bytes
+  __device__ __forceinline__ uint32_t s_free(int h) const { return base + 8u * (2 * NS + 16 + h); }
+  static constexpr uint32_t kItemsOff = 8u * (2 * NS + 18);  // 2 x 40 bytes
   static constexpr uint32_t kTmemOff = kItemsOff + 96;
   static constexpr uint32_t kAbortOff = kTmemOff + 8;
   static constexpr uint32_t kBadWsOff = kAbortOff + 8;
@@ -136,6 +145,45 @@ __device__ __noinline__ void drain_bar(uint32_t a, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(a, parity))
     if (globaltimer_ns() - t0 > 200000000ull) return;
+}
+
+// O_h *= alpha in TMEM, 32 columns at a time (one thread per row).
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int q = 0; q < D / 32; ++q) {
+    uint32_t o[32];
+    tmem_ld32(tO + q * 32, o);
+    tmem_ld_wait();
+    tmem_ld_fence32(o);
+#pragma unroll
+    for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+    tmem_st32(tO + q * 32, o);
+  }
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Makes this thread's shared-memory stores visible to the tensor core (the async proxy).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One P row (BK bf16, packed in pairs in r[0, BK/2)) into a K-major 128-byte-swizzle tile of
+// 128 rows: keys [64c, 64c + 64) in chunk c (128 rows x 128 bytes), row lr at byte lr * 128 of the
+// chunk, its 16-byte unit u at position u ^ (lr % 8). A warp's 32 rows cover all banks in four
+// passes per store.
+template <int BK>
+__device__ __forceinline__ void store_p_sw128(uint32_t base, int lr, const uint32_t* r) {
+  const uint32_t row = base + (uint32_t)lr * 128u, sw = (uint32_t)lr & 7u;
+#pragma unroll
+  for (int ch = 0; ch < BK / 64; ++ch)
+#pragma unroll
+    for (uint32_t u = 0; u < 8; ++u) {
+      const uint32_t* w = r + ch * 32 + 4 * u;
+      st_shared_v4(row + ch * (128u * 128u) + ((u ^ sw) << 4), w[0], w[1], w[2], w[3]);
+    }
 }
 
 template <int BK>
@@ -183,9 +231,9 @@ __device__ ItemInfo decode_item(const AttnParams& P, uint32_t idx) {
 }
 
 // ---------------------------------------------------------------------------------------
-template <int D, int BK, bool QK8 = false>
+template <int D, int BK, bool QK8 = false, bool PS = false>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
-  using C = Cfg<D, BK, QK8>;
+  using C = Cfg<D, BK, QK8, PS>;
   constexpr int NS = C::kStages;
   using K = Ctl<NS>;
   static_assert(K::kBytes <= 1024, "control block");
@@ -193,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   // 1024-byte alignment for the 128-byte swizzle atoms
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = raw + ((1024u - (raw & 1023u)) & 1023u);
-  const uint32_t sQ = sbase, sRing = sbase + C::kQBytes;
+  const uint32_t sQ = sbase, sP = sbase + C::kQBytes, sRing = sP + C::kPBytes;
   K c;
   c.base = sbase + C::kDataBytes;
   c.status = P.status;
@@ -221,6 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     mbar_init(b + 14, 1);  // drain
     mbar_init(b + 15, 1);  // never
+    mbar_init(b + 16, 128);  // s_free[0]
+    mbar_init(b + 17, 128);  // s_free[1]
     *reinterpret_cast<volatile int*>(ctl_gen + K::kAbortOff) = 0;
     // the tile maps must have been built for exactly these parameters
     int bad = 0;
@@ -301,8 +351,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         q_issued = true;
       }
+      // K / V loads in the order the MMA warp consumes them: K(e), V(e) per entry; with P in
+      // shared memory S(e+1) comes before P V(e): K(0), then K(e+1), V(e) per entry.
       bool ok = true;
-      for (int e = 0; e < inf.count && ok; ++e) {
+      for (int n = 0; n < 2 * inf.count && ok; ++n) {
+        int e, w;
+        if (!PS) {
+          e = n >> 1;
+          w = n & 1;
+        } else if (n == 0) {
+          e = 0;
+          w = 0;
+        } else if (n == 2 * inf.count - 1) {
+          e = inf.count - 1;
+          w = 1;
+        } else {
+          const int m = n - 1;
+          e = (m >> 1) + ((m & 1) ^ 1);
+          w = m & 1;
+        }
         const uint32_t ent = get_entry<BK>(P, inf, e);
         const int row0 = (int)ent_kt(ent) * BK;
         int rr[4] = {0, 0, 0, 0};
@@ -310,32 +377,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
           for (int i = 0; i < 4; ++i) rr[i] = hrow + orig_index(gg, min(row0 + 4 * lane + i, P.N - 1));
         }
-        for (int w = 0; w < 2; ++w) {
-          const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
-          if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status) : 0,
-                           0)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) mbar_expect_tx(c.kv_full(st), w == 0 ? C::kKBytes : C::kVBytes);
-          __syncwarp();
-          const uint32_t dst = sRing + st * C::kTileBytes;
-          if (gat) {
-            if (4 * lane < BK)
-              for (int ch = 0; ch < C::kChunks; ++ch)
-                tma_gather4(dst + ch * (BK * 128) + lane * 512, w == 0 ? &P.tm_k2 : &P.tm_v2, c.kv_full(st), ch * 64,
-                            rr[0], rr[1], rr[2], rr[3]);
-          } else if (lane == 0) {
-            if (w == 0) {
-              for (int ch = 0; ch < C::kQKChunks; ++ch)
-                tma_load_3d(dst + ch * (BK * 128), &P.tm_k, c.kv_full(st), ch * C::kQKColsPerChunk, row0, inf.head);
-            } else {
-              for (int ch = 0; ch < C::kChunks; ++ch)
-                tma_load_3d(dst + ch * (BK * 128), &P.tm_v, c.kv_full(st), ch * 64, row0, inf.head);
-            }
-          }
-          ++kv_pos;
+        const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
+        if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status) : 0,
+                         0)) {
+          ok = false;
+          break;
         }
+        if (lane == 0) mbar_expect_tx(c.kv_full(st), w == 0 ? C::kKBytes : C::kVBytes);
+        __syncwarp();
+        const uint32_t dst = sRing + st * C::kTileBytes;
+        if (gat) {
+          if (4 * lane < BK)
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tma_gather4(dst + ch * (BK * 128) + lane * 512, w == 0 ? &P.tm_k2 : &P.tm_v2, c.kv_full(st), ch * 64,
+                          rr[0], rr[1], rr[2], rr[3]);
+        } else if (lane == 0) {
+          if (w == 0) {
+            for (int ch = 0; ch < C::kQKChunks; ++ch)
+              tma_load_3d(dst + ch * (BK * 128), &P.tm_k, c.kv_full(st), ch * C::kQKColsPerChunk, row0, inf.head);
+          } else {
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tma_load_3d(dst + ch * (BK * 128), &P.tm_v, c.kv_full(st), ch * 64, row0, inf.head);
+          }
+        }
+        ++kv_pos;
       }
       if (!ok) break;
     }
@@ -358,9 +423,119 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       const uint64_t qdesc = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t kdesc = smem_desc_sw128(sRing, 16, 1024);
       const uint64_t vdesc = smem_desc_sw128(sRing, BK * 128, 1024);
+      // S_h = Q_h K^T from the K tile at descriptor kd, then s_full[h]
+      auto issue_s = [&](int h, uint64_t kd) {
+        const uint64_t qd = qdesc + ((h * C::kQHalfBytes) >> 4);
+        if constexpr (QK8) {
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk) {
+            // 32 e4m3 = 32 bytes along K inside a 128-byte swizzle atom; 128 columns per atom
+            const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+            const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
+            umma_ss_f8(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // 16 bf16 = 32 bytes along K inside a 128-byte swizzle atom; 64 columns per atom
+            const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+            const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
+            umma_ss(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(c.s_full(h));
+      };
       uint32_t kv_pos = 0, q_iter = 0, p_cnt0 = 0, p_cnt1 = 0, of_cnt0 = 0, of_cnt1 = 0;
       bool ok = true;
-      for (uint32_t it = 0; ok; ++it) {
+      if constexpr (PS) {
+        // P in shared memory. Per entry e: S_h(e+1) as soon as the softmax has loaded S_h(e)
+        // (s_free), then O_h += P_h(e) V(e) once P_h(e) is stored (p_ready); every P V commits
+        // pv_done[h] (the o_done barrier), which frees P_h's buffer and orders O_h for the softmax.
+        const uint64_t pdesc = smem_desc_sw128(sP, 16, 1024);
+        uint32_t sf_cnt0 = 0, sf_cnt1 = 0;
+        // S(e) of the entry's active halves from ring position kpos, then the K slot's release
+        auto s_entry = [&](uint32_t ent, uint32_t kpos, bool last_s) -> bool {
+          bool k_ready = false;
+          const uint64_t kd = kdesc + (((kpos % NS) * C::kTileBytes) >> 4);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (ent_flag(ent, h) == kFlagSkip) continue;
+            uint32_t& sc = h == 0 ? sf_cnt0 : sf_cnt1;
+            if (sc > 0 && !wait_bar(c.s_free(h), (sc - 1) & 1u, abort_addr, status)) return false;
+            ++sc;
+            if (!k_ready) {
+              if (!wait_bar(c.kv_full(kpos % NS), (kpos / NS) & 1u, abort_addr, status)) return false;
+              k_ready = true;
+            }
+            tc_fence_after();  // after the softmax's loads of the previous S_h
+            issue_s(h, kd);
+          }
+          if (!k_ready && !wait_bar(c.kv_full(kpos % NS), (kpos / NS) & 1u, abort_addr, status)) return false;
+          umma_commit(c.kv_empty(kpos % NS));  // K read by the S MMAs
+          if (last_s) umma_commit(c.q_free());  // Q read by the item's last S MMA
+          return true;
+        };
+        for (uint32_t it = 0; ok; ++it) {
+          const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
+          if (!wait_bar(c.item_full(slot), ph, abort_addr, status)) break;
+          const ItemInfo inf = items[slot];
+          mbar_arrive(c.item_empty(slot));
+          if (!inf.valid) break;
+          if (inf.nA + inf.nB > 0) {
+            if (!wait_bar(c.q_full(), q_iter & 1u, abort_addr, status)) break;
+            ++q_iter;
+          }
+          uint32_t has_o = 0;
+          uint32_t ent_n = inf.count > 0 ? get_entry<BK>(P, inf, 0) : 0u;
+          if (inf.count > 0) ok = s_entry(ent_n, kv_pos++, inf.count == 1);
+          for (int e = 0; e < inf.count && ok; ++e) {
+            const uint32_t ent = ent_n;
+            if (e + 1 < inf.count) {
+              ent_n = get_entry<BK>(P, inf, e + 1);
+              ok = s_entry(ent_n, kv_pos++, e + 2 == inf.count);
+              if (!ok) break;
+            }
+            const uint32_t vpos = kv_pos++;
+            bool v_ready = false;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (ent_flag(ent, h) == kFlagSkip) continue;
+              uint32_t& pc = h == 0 ? p_cnt0 : p_cnt1;
+              uint32_t& oc = h == 0 ? of_cnt0 : of_cnt1;
+              ok = wait_bar(c.p_ready(h), pc & 1u, abort_addr, status);
+              ++pc;
+              if (ok && !((has_o >> h) & 1u)) {
+                ok = wait_bar(c.o_free(h), (oc & 1u) ^ 1u, abort_addr, status);
+                ++oc;
+              }
+              if (ok && !v_ready) {
+                ok = wait_bar(c.kv_full(vpos % NS), (vpos / NS) & 1u, abort_addr, status);
+                v_ready = true;
+              }
+              if (!ok) break;
+              tc_fence_after();
+              const uint64_t vd = vdesc + (((vpos % NS) * C::kTileBytes) >> 4);
+              const uint64_t pd = pdesc + ((h * C::kPHalfBytes) >> 4);
+              const uint32_t acc0 = (has_o >> h) & 1u;
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint32_t poff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                umma_ss(tmem + C::o_col(h), pd + poff, vd + ((kk * 2048) >> 4), idesc_o,
+                        (acc0 || kk > 0) ? 1u : 0u);
+              }
+              umma_commit(c.o_done(h));
+              has_o |= 1u << h;
+            }
+            if (!ok) break;
+            if (!v_ready) {
+              ok = wait_bar(c.kv_full(vpos % NS), (vpos / NS) & 1u, abort_addr, status);
+              if (!ok) break;
+            }
+            umma_commit(c.kv_empty(vpos % NS));  // V read by the P V MMAs
+          }
+        }
+      }
+      for (uint32_t it = 0; ok && !PS; ++it) {
         const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
         if (!wait_bar(c.item_full(slot), ph, abort_addr, status)) break;
         const ItemInfo inf = items[slot];
@@ -413,25 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 if (!ok) break;
                 k_ready = true;
               }
-              const uint64_t qd = qdesc + ((h * C::kQHalfBytes) >> 4);
-              if constexpr (QK8) {
-#pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk) {
-                  // 32 e4m3 = 32 bytes along K inside a 128-byte swizzle atom; 128 columns per atom
-                  const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
-                  const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
-                  umma_ss_f8(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
-                }
-              } else {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                  // 16 bf16 = 32 bytes along K inside a 128-byte swizzle atom; 64 columns per atom
-                  const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
-                  const uint32_t koff = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
-                  umma_ss(tmem + C::s_col(h), qd + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
-                }
-              }
-              umma_commit(c.s_full(h));
+              issue_s(h, kd);
             }
             prev_act = (prev_act & ~(1u << h)) | ((act ? 1u : 0u) << h);
           }
@@ -461,8 +618,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const uint32_t tS = tmem + lane_off + C::s_col(h);
     const uint32_t tP = tS + C::kPCol;
     const uint32_t tO = tmem + lane_off + C::o_col(h);
+    const uint32_t sPh = sP + h * C::kPHalfBytes;
     const float sl2 = P.sl2;
-    uint32_t s_cnt = 0, od_cnt = 0;
+    uint32_t s_cnt = 0, od_cnt = 0, pv_cnt = 0;
     // (test hook) a wait that nothing satisfies: it gives up after the limit, raises the abort
     // flag and the timeout status, and every role drains and leaves
     const bool stalled = P.inject_stall && !__all_sync(0xffffffffu, wait_bar(c.never(), 0, abort_addr, status));
@@ -517,33 +675,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         float alpha = 1.f;
         float2 acc[2];
         load_scores<BK>(tS, r);
+        if constexpr (PS) {  // S_h's columns are free for the next tile's S_h
+          tc_fence_before();
+          mbar_arrive(c.s_free(h));
+        }
         mask_scores<BK>(P, inf.cls, f, c0, prow, ent, lo, hi, se, per, r);
         const bool rescale = max_first<BK>(r, sl2, m, l, alpha);
         exp_tile<BK>(r, sl2, m, acc);
         l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
-#pragma unroll
-        for (int q = 0; q < BK / 64; ++q) tmem_st32(tP + q * 32, r + q * 32);
-        if (rescale && !first) {  // O_h holds every earlier P V (S_h's commit covered them)
-#pragma unroll 1
-          for (int q = 0; q < D / 32; ++q) {
-            uint32_t o[32];
-            tmem_ld32(tO + q * 32, o);
-            tmem_ld_wait();
-            tmem_ld_fence32(o);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tO + q * 32, o);
+        if constexpr (PS) {
+          // the previous P_h V is complete: P_h's buffer is free and O_h holds every earlier P V
+          if (pv_cnt > 0 &&
+              !__all_sync(0xffffffffu, wait_bar(c.o_done(h), (pv_cnt - 1) & 1u, abort_addr, status))) {
+            ok = false;
+            break;
           }
+          ++pv_cnt;
+          if (rescale && !first) {
+            tc_fence_after();
+            rescale_o<D>(tO, alpha);
+            tmem_st_wait();
+          }
+          store_p_sw128<BK>(sPh, lr, r);
+          fence_proxy_async_shared();
+          tc_fence_before();
+          mbar_arrive(c.p_ready(h));
+        } else {
+#pragma unroll
+          for (int q = 0; q < BK / 64; ++q) tmem_st32(tP + q * 32, r + q * 32);
+          if (rescale && !first) rescale_o<D>(tO, alpha);  // O_h holds every earlier P V (S_h's commit covered them)
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(c.p_ready(h));
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(c.p_ready(h));
         first = false;
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16
-      if (!__all_sync(0xffffffffu, wait_bar(c.o_done(h), od_cnt & 1u, abort_addr, status))) break;
-      ++od_cnt;
+      if constexpr (PS) {
+        if (!__all_sync(0xffffffffu, wait_bar(c.o_done(h), (pv_cnt - 1) & 1u, abort_addr, status))) break;
+      } else {
+        if (!__all_sync(0xffffffffu, wait_bar(c.o_done(h), od_cnt & 1u, abort_addr, status))) break;
+        ++od_cnt;
+      }
       tc_fence_after();
       const float inv_l = (l > 0.f && m != -INFINITY) ? 1.f / l : 0.f;  // a row with no kept key gives 0
       __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + orow_idx) * D;
@@ -581,10 +755,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------------------------------
-template <int D, int BK, bool QK8 = false>
+template <int D, int BK, bool QK8, bool PS>
 static int launch_t(const AttnParams& P, int grid, cudaStream_t st) {
-  using C = Cfg<D, BK, QK8>;
-  auto kern = attn_kernel<D, BK, QK8>;
+  using C = Cfg<D, BK, QK8, PS>;
+  auto kern = attn_kernel<D, BK, QK8, PS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return record_cuda_error("cudaFuncSetAttribute(attn_kernel)", e);
   kern<<<grid, kThreads, C::kSmemBytes, st>>>(P);
@@ -592,17 +766,23 @@ static int launch_t(const AttnParams& P, int grid, cudaStream_t st) {
   return e == cudaSuccess ? SVG_OK : record_cuda_error("launch attn_kernel", e);
 }
 
-int launch_attention(const AttnParams& P, int d, int bk, int grid, cudaStream_t st) {
+template <bool PS>
+static int launch_ps(const AttnParams& P, int d, int bk, int grid, cudaStream_t st) {
   if (P.qk8) {  // e4m3 Q and K: d = 128
-    if (d == 128 && bk == 128) return launch_t<128, 128, true>(P, grid, st);
-    if (d == 128 && bk == 64) return launch_t<128, 64, true>(P, grid, st);
+    if (d == 128 && bk == 128) return launch_t<128, 128, true, PS>(P, grid, st);
+    if (d == 128 && bk == 64) return launch_t<128, 64, true, PS>(P, grid, st);
     return SVG_ERR_UNSUPPORTED;
   }
-  if (d == 128 && bk == 128) return launch_t<128, 128>(P, grid, st);
-  if (d == 128 && bk == 64) return launch_t<128, 64>(P, grid, st);
-  if (d == 64 && bk == 128) return launch_t<64, 128>(P, grid, st);
-  if (d == 64 && bk == 64) return launch_t<64, 64>(P, grid, st);
+  if (d == 128 && bk == 128) return launch_t<128, 128, false, PS>(P, grid, st);
+  if (d == 128 && bk == 64) return launch_t<128, 64, false, PS>(P, grid, st);
+  if (d == 64 && bk == 128) return launch_t<64, 128, false, PS>(P, grid, st);
+  if (d == 64 && bk == 64) return launch_t<64, 64, false, PS>(P, grid, st);
   return SVG_ERR_UNSUPPORTED;
+}
+
+// p_smem: P staged in shared memory (the decoupled schedule) instead of TMEM.
+int launch_attention(const AttnParams& P, int d, int bk, int grid, bool p_smem, cudaStream_t st) {
+  return p_smem ? launch_ps<true>(P, d, bk, grid, st) : launch_ps<false>(P, d, bk, grid, st);
 }
 
 size_t attn_params_size() { return sizeof(AttnParams); }

@@ -41,7 +41,8 @@
  *     SVG_ERR_UNSUPPORTED.
  *   - Environment (read by the host code): SVG_KERNEL=pair or SVG_KERNEL=pair1 (read once per
  *     process) makes d = 128 attention run on the two-SM kernels instead of the one-SM kernel,
- *     with the same results up to rounding; SVG_TEST_STALL=1 (read on every call) is a test hook
+ *     and SVG_KERNEL=ps makes the one-SM kernel stage P in shared memory instead of tensor
+ *     memory, each with the same results up to rounding; SVG_TEST_STALL=1 (read on every call) is a test hook
  *     that makes an attention launch wait on a barrier nothing completes, so that it ends with
  *     SVG_ERR_TIMEOUT in its status word after the wait limit (2 s).
  */

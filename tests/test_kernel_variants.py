@@ -1,5 +1,6 @@
-"""The selectable two-SM kernels (SVG_KERNEL=pair: 512-row items, two halves per SM; SVG_KERNEL=pair1:
-one 128-row half per SM, key tiles alternating between two softmax groups) against the oracle.
+"""The selectable kernels (SVG_KERNEL=pair: 512-row items, two halves per SM; SVG_KERNEL=pair1:
+one 128-row half per SM, key tiles alternating between two softmax groups; SVG_KERNEL=ps: the
+single-SM kernel with P staged in shared memory) against the oracle.
 The kernel choice is read once per process, so each runs in a child process."""
 import os
 import subprocess
@@ -40,7 +41,7 @@ print("ok")
 """
 
 
-@pytest.mark.parametrize("kernel", ["pair", "pair1"])
+@pytest.mark.parametrize("kernel", ["pair", "pair1", "ps"])
 def test_two_sm_kernels_match_oracle(kernel):
     env = dict(os.environ, SVG_KERNEL=kernel)
     r = subprocess.run([sys.executable, "-c", CHILD.format(root=ROOT)], env=env, cwd=ROOT, capture_output=True,
