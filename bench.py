@@ -225,6 +225,8 @@ def main():
     ap.add_argument("--quick", action="store_true",
                     help="only the timed steps (no side measurements, e2e or CPU baseline): for profiler runs")
     ap.add_argument("--heads", type=int, default=0, help="use only the first H heads of the workload")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="split one call's heads over the ranks (strong scaling) instead of running replicas")
     ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=96, help="oracle rows per head per --impl reference step")
     args = ap.parse_args()
@@ -255,6 +257,22 @@ def main():
     mode = S.SVG_MODE_SPLIT if args.mode == "split" else S.SVG_MODE_NAIVE
 
     q_cpu, k_cpu, v_cpu = syn.make_qkv(w)
+    ws = [None, None]
+    summ = [None, None]
+    for c in sorted(set(routes)):
+        ws[c] = S.alloc_workspace(g, t, dev)
+        S.svg_build_tilemap(g, m, t, c, ws[c])
+        summ[c] = S.svg_tilemap_summary(ws[c])
+    plan = None
+    if args.shard_heads:
+        # one call's heads split over the ranks by tile-map work; each rank keeps only its heads
+        from block_sparse_spatio_flash_b200 import shard
+        if world > w.heads:
+            raise SystemExit(f"--shard-heads needs at least one head per rank ({w.heads} heads, {world} ranks)")
+        plan = shard.plan_heads(shard.head_costs(routes, summ), world)
+        q_cpu, k_cpu, v_cpu = (shard.local_heads(x, plan, rank) for x in (q_cpu, k_cpu, v_cpu))
+        w = w.replace(routes=tuple(shard.local_routes(plan, rank, routes)))
+        routes = list(w.routes)
     q, k, v = (x.to(dev) for x in (q_cpu, k_cpu, v_cpu))
     if any(routes):  # temporal heads run in their own token order (permutation timed separately)
         qp, kp, vp = (torch.empty_like(x) for x in (q, k, v))
@@ -264,17 +282,15 @@ def main():
         qp, kp, vp = q, k, v
     o = torch.empty_like(qp)
     scratch = S.alloc_scratch(dev)
-
-    ws = [None, None]
-    summ = [None, None]
-    for c in sorted(set(routes)):
-        ws[c] = S.alloc_workspace(g, t, dev)
-        S.svg_build_tilemap(g, m, t, c, ws[c])
-        summ[c] = S.svg_tilemap_summary(ws[c])
     eff_flop, vis_flop, exe_flop = workload_flops(w, summ)
+    o_all = None
+    if plan is not None and world > 1:
+        o_all = torch.empty((plan.heads,) + tuple(o.shape[1:]), dtype=o.dtype, device=dev)
 
     def step():
         S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, mode=mode, scratch=scratch)
+        if o_all is not None:  # every rank ends the step with all heads' O
+            shard.gather_heads(o, plan, out=o_all)
 
     for _ in range(args.warmup):
         step()
@@ -338,12 +354,13 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong" if plan is not None else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d,
                        "routes": "".join("S" if r == 0 else "T" for r in routes),
                        "frame_window": w.frame_window, "spatial_band": w.spatial_band, "sink_frames": w.sink_frames,
-                       "bq": w.bq, "bk": w.bk, "mode": args.mode, "parallelism": f"replicas x{world}",
+                       "bq": w.bq, "bk": w.bk, "mode": args.mode, "parallelism": (f"heads x{world} (all-gather of O in the step)" if plan is not None
+                                       else f"replicas x{world}"),
                        "l2": "no flush: Q/K/V/O = %.0f MB > 126 MB L2" % (4 * w.heads * w.tokens * w.d * 2 / 1e6)},
             "ms_per_call": ms,
             "effective_flop_per_call": eff_flop, "visited_flop_per_call": vis_flop, "executed_flop_per_call": exe_flop,
