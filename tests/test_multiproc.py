@@ -33,7 +33,7 @@ def _worker(rank, world, port, out):
 def test_aggregate_over_ranks_gloo():
     world = 2
     port = _free_port()
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)

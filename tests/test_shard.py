@@ -95,7 +95,7 @@ def _gather_worker(rank, world, port, costs, out):
                                          (3, [3, 8, 2, 7, 7, 1, 0, 4]), (3, [1, 1])])
 def test_gather_heads_gloo(world, costs):
     port = _free_port()
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.spawn(_gather_worker, args=(world, port, costs, out), nprocs=world, join=True)
         res = dict(out)
@@ -138,7 +138,7 @@ def _oracle_worker(rank, world, port, out):
 def test_sharded_heads_keep_their_routes_gloo():
     world = 2
     port = _free_port()
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.spawn(_oracle_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
