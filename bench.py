@@ -336,7 +336,7 @@ def main():
     e2e = None
     if not args.quick:
         e2e = end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream,
-                         args)
+                         args, attn_ms=statistics.mean(per_step))
 
     cpu = None
     if rank == 0 and world == 1 and not args.quick:
@@ -547,7 +547,8 @@ def other_workloads(S, P, stream, dev):
     return res
 
 
-def end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream, args):
+def end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, eff_flop, world, dev, stream, args,
+               attn_ms=None):
     """Same metric through the public C-ABI call on host buffers (svg_attention_fwd_host): every
     step copies Q/K/V in from pinned host memory, permutes temporal heads, runs the attention,
     permutes O back and copies it out, in chunks of heads whose copies overlap the neighbouring
@@ -576,9 +577,21 @@ def end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, ef
     ms, value = aggregate_over_ranks(ms_local, eff_flop, world, dev)
     h2d = 3 * q_cpu.numel() * 2
     d2h = q_cpu.numel() * 2
-    return {"value": value, "unit": "TFLOP/s", "ms_per_step": ms, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": n, "call": "svg_attention_fwd_host", "chunk_heads": ch,
-            "clock": "host, between device synchronisations"}
+    out = {"value": value, "unit": "TFLOP/s", "ms_per_step": ms, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": n, "call": "svg_attention_fwd_host", "chunk_heads": ch,
+           "clock": "host, between device synchronisations"}
+    # the copies alone, one direction at a time (pinned host memory, one copy per tensor): the pipeline
+    # cannot beat all of H2D plus the last chunk's attention and D2H
+    dq = [torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (qh, kh, vh)]
+    h2d_ms = time_events(lambda: [d.copy_(x, non_blocking=True) for d, x in zip(dq, (qh, kh, vh))], 3, stream)
+    d2h_ms = time_events(lambda: oh.copy_(dq[0], non_blocking=True), 3, stream)
+    out.update(h2d_ms=h2d_ms, h2d_gbs=h2d / h2d_ms / 1e6, d2h_ms=d2h_ms, d2h_gbs=d2h / d2h_ms / 1e6)
+    if attn_ms is not None:
+        chunks = -(-w.heads // ch)
+        bound = h2d_ms + (attn_ms + d2h_ms) / chunks
+        out.update(copy_bound_ms=bound, frac_of_copy_bound=bound / ms)
+    del dq
+    return out
 
 
 if __name__ == "__main__":
