@@ -353,6 +353,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       // K / V loads in the order the MMA warp consumes them: K(e), V(e) per entry; with P in
       // shared memory S(e+1) comes before P V(e): K(0), then K(e+1), V(e) per entry.
+      // the last two entries' key-tile row and gathered row indices, {entry, row0, rr[4]} by entry
+      // parity: each entry's are worked out once (static indices only, so they stay in registers)
+      int ca[6] = {-1, 0, 0, 0, 0, 0}, cb[6] = {-1, 0, 0, 0, 0, 0};
+      auto fill = [&](int (&cc)[6], int e) {
+        cc[0] = e;
+        cc[1] = (int)ent_kt(get_entry<BK>(P, inf, e)) * BK;
+        if (gat && 4 * lane < BK) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cc[2 + i] = hrow + orig_index(gg, min(cc[1] + 4 * lane + i, P.N - 1));
+        }
+      };
       bool ok = true;
       for (int n = 0; n < 2 * inf.count && ok; ++n) {
         int e, w;
@@ -370,12 +381,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           e = (m >> 1) + ((m & 1) ^ 1);
           w = m & 1;
         }
-        const uint32_t ent = get_entry<BK>(P, inf, e);
-        const int row0 = (int)ent_kt(ent) * BK;
-        int rr[4] = {0, 0, 0, 0};
-        if (gat && 4 * lane < BK) {
+        int row0, rr[4];
+        if ((e & 1) == 0) {
+          if (ca[0] != e) fill(ca, e);
+          row0 = ca[1];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) rr[i] = hrow + orig_index(gg, min(row0 + 4 * lane + i, P.N - 1));
+          for (int i = 0; i < 4; ++i) rr[i] = ca[2 + i];
+        } else {
+          if (cb[0] != e) fill(cb, e);
+          row0 = cb[1];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) rr[i] = cb[2 + i];
         }
         const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
         if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status) : 0,
