@@ -586,9 +586,26 @@ def end_to_end(S, w, g, m, t, routes, q_cpu, k_cpu, v_cpu, ws, scratch, mode, ef
     h2d_ms = time_events(lambda: [d.copy_(x, non_blocking=True) for d, x in zip(dq, (qh, kh, vh))], 3, stream)
     d2h_ms = time_events(lambda: oh.copy_(dq[0], non_blocking=True), 3, stream)
     out.update(h2d_ms=h2d_ms, h2d_gbs=h2d / h2d_ms / 1e6, d2h_ms=d2h_ms, d2h_gbs=d2h / d2h_ms / 1e6)
+    # both directions at once, as in the pipeline: all inputs in on one stream while as many bytes as the
+    # outputs go out on another; the link is shared, so this time bounds the pipeline too
+    side = torch.cuda.Stream(device=dev)
+    ev0, ev1, ev2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    side.wait_event(ev0)
+    with torch.cuda.stream(side):
+        oh.copy_(dq[0], non_blocking=True)
+        ev2.record(side)
+    for d_, x in zip(dq, (qh, kh, vh)):
+        d_.copy_(x, non_blocking=True)
+    stream.wait_event(ev2)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    duplex_ms = ev0.elapsed_time(ev1)
+    out.update(duplex_ms=duplex_ms, duplex_gbs=(h2d + d2h) / duplex_ms / 1e6)
     if attn_ms is not None:
         chunks = -(-w.heads // ch)
-        bound = h2d_ms + (attn_ms + d2h_ms) / chunks
+        bound = max(h2d_ms + (attn_ms + d2h_ms) / chunks, duplex_ms)
         out.update(copy_bound_ms=bound, frac_of_copy_bound=bound / ms)
     del dq
     return out
