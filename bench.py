@@ -179,6 +179,14 @@ def closed_form_effective_flops(w):
     return 4 * w.d * tot
 
 
+def workload_config(w, args, parallelism, l2):
+    """The `config` object of both arms' JSON lines: the workload and the launch shape."""
+    return {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d,
+            "routes": "".join("S" if r == 0 else "T" for r in w.routes),
+            "frame_window": w.frame_window, "spatial_band": w.spatial_band, "sink_frames": w.sink_frames,
+            "bq": w.bq, "bk": w.bk, "mode": args.mode, "parallelism": parallelism, "l2": l2}
+
+
 def run_reference(args, w, world, rank):
     if rank != 0:
         return 0
@@ -199,7 +207,8 @@ def run_reference(args, w, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d},
+        "config": workload_config(w, args, f"oracle on the host cores of rank 0 of {world}",
+                                  "n/a (host memory)"),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
                          "sample": f"{rows} seeded query rows per head x {w.heads} heads per step; full-call time = "
                                    f"once-per-head part ({fixed:.2f} s, timed with one row per head) + per-row "
@@ -356,12 +365,9 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong" if plan is not None else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d,
-                       "routes": "".join("S" if r == 0 else "T" for r in routes),
-                       "frame_window": w.frame_window, "spatial_band": w.spatial_band, "sink_frames": w.sink_frames,
-                       "bq": w.bq, "bk": w.bk, "mode": args.mode, "parallelism": (f"heads x{world} (all-gather of O in the step)" if plan is not None
-                                       else f"replicas x{world}"),
-                       "l2": "no flush: Q/K/V/O = %.0f MB > 126 MB L2" % (4 * w.heads * w.tokens * w.d * 2 / 1e6)},
+            "config": workload_config(
+                w, args, f"heads x{world} (all-gather of O in the step)" if plan is not None else f"replicas x{world}",
+                "no flush: Q/K/V/O = %.0f MB > 126 MB L2" % (4 * w.heads * w.tokens * w.d * 2 / 1e6)),
             "ms_per_call": ms,
             "effective_flop_per_call": eff_flop, "visited_flop_per_call": vis_flop, "executed_flop_per_call": exe_flop,
             "visited_tflops": vis_flop / (ms * 1e-3) / 1e12,
