@@ -333,7 +333,7 @@ def main():
     achieved = vis_flop / (statistics.mean(per_step) * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": captured_traffic(w, args),
-                "kernel": "attn_kernel<128,128> (split)", "flop_definition": "4*d*(in-range area of visited tiles)",
+                "kernel": f"attn_kernel<128,128> ({args.mode}, {kernel_variant()} schedule)", "flop_definition": "4*d*(in-range area of visited tiles)",
                 "peak_kind": f"{peak_kind} bf16 burst"}
 
     extras = {}
@@ -398,10 +398,15 @@ def kernel_sources_sha() -> str:
     return h.hexdigest()[:16]
 
 
+def kernel_variant() -> str:
+    """The attention kernel the library runs: its default, or the option named by SVG_KERNEL."""
+    return os.environ.get("SVG_KERNEL", "") or "default"
+
+
 def captured_traffic(w, args):
     c = CAPTURED_TRAFFIC
     if (kernel_sources_sha() != c["sources_sha256"] or w.name != c["workload"] or args.bq != c["bq"]
-            or args.bk != c["bk"] or args.mode != c["mode"]):
+            or args.bk != c["bk"] or args.mode != c["mode"] or kernel_variant() != "default"):
         return None
     return c["bytes_per_head"] * w.heads
 

@@ -15,6 +15,7 @@ def _args(**kw):
 
 def test_traffic_only_for_the_captured_kernel_and_workload(monkeypatch):
     c = bench.CAPTURED_TRAFFIC
+    monkeypatch.delenv("SVG_KERNEL", raising=False)
     w = syn.WORKLOADS[c["workload"]]
     monkeypatch.setattr(bench, "kernel_sources_sha", lambda: c["sources_sha256"])
     assert bench.captured_traffic(w, _args()) == c["bytes_per_head"] * w.heads
@@ -25,6 +26,11 @@ def test_traffic_only_for_the_captured_kernel_and_workload(monkeypatch):
     assert bench.captured_traffic(w, _args(bk=64)) is None
     assert bench.captured_traffic(w, _args(mode="naive")) is None
     assert bench.captured_traffic(syn.TINY, _args()) is None
+    # another kernel option selected: no figure
+    monkeypatch.setenv("SVG_KERNEL", "ps")
+    assert bench.captured_traffic(w, _args()) is None
+    monkeypatch.delenv("SVG_KERNEL")
+    assert bench.captured_traffic(w, _args()) == c["bytes_per_head"] * w.heads
     # changed kernel sources: no figure
     monkeypatch.setattr(bench, "kernel_sources_sha", lambda: "0" * 16)
     assert bench.captured_traffic(w, _args()) is None
