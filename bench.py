@@ -333,8 +333,8 @@ def main():
     achieved = vis_flop / (statistics.mean(per_step) * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": captured_traffic(w, args),
-                "kernel": f"attn_kernel<128,128> ({args.mode}, {kernel_variant()} schedule)", "flop_definition": "4*d*(in-range area of visited tiles)",
-                "peak_kind": f"{peak_kind} bf16 burst"}
+                "kernel": f"attn_kernel<128,128> ({args.mode}, {kernel_variant()} schedule)",
+                "flop_definition": "4*d*(in-range area of visited tiles)", "peak_kind": f"{peak_kind} bf16 burst"}
 
     extras = {}
     if not (args.no_extras or args.quick):
