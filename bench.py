@@ -62,14 +62,16 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, log_dir: str = ""):
+        import tempfile
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = os.path.join(log_dir or tempfile.gettempdir(), f"svg_bench_clocks_rank{device_index}.csv")
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            if os.path.dirname(self.path):
+                os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
@@ -179,12 +181,14 @@ def closed_form_effective_flops(w):
     return 4 * w.d * tot
 
 
-def workload_config(w, args, parallelism, l2):
-    """The `config` object of both arms' JSON lines: the workload and the launch shape."""
+def workload_config(w, args):
+    """The `config` object of both arms' JSON lines: the workload and the launch shape only, so that
+    the two arms print identical objects; how the work is spread and the cache policy are top-level
+    keys of the line."""
     return {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d,
             "routes": "".join("S" if r == 0 else "T" for r in w.routes),
             "frame_window": w.frame_window, "spatial_band": w.spatial_band, "sink_frames": w.sink_frames,
-            "bq": w.bq, "bk": w.bk, "mode": args.mode, "parallelism": parallelism, "l2": l2}
+            "bq": w.bq, "bk": w.bk, "mode": args.mode}
 
 
 def run_reference(args, w, world, rank):
@@ -207,8 +211,8 @@ def run_reference(args, w, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args, f"oracle on the host cores of rank 0 of {world}",
-                                  "n/a (host memory)"),
+        "config": workload_config(w, args),
+        "parallelism": f"oracle on the host cores of rank 0 of {world}", "l2": "n/a (host memory)",
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
                          "sample": f"{rows} seeded query rows per head x {w.heads} heads per step; full-call time = "
                                    f"once-per-head part ({fixed:.2f} s, timed with one row per head) + per-row "
@@ -238,6 +242,8 @@ def main():
                     help="split one call's heads over the ranks (strong scaling) instead of running replicas")
     ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=96, help="oracle rows per head per --impl reference step")
+    ap.add_argument("--clock-log-dir", default="",
+                    help="folder for the nvidia-smi clock samples of the timed region (default: the temp folder)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -310,7 +316,7 @@ def main():
 
     # ---------------------------------------------------------------- timed region
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, args.clock_log_dir) as clk:
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -365,9 +371,9 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong" if plan is not None else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(
-                w, args, f"heads x{world} (all-gather of O in the step)" if plan is not None else f"replicas x{world}",
-                "no flush: Q/K/V/O = %.0f MB > 126 MB L2" % (4 * w.heads * w.tokens * w.d * 2 / 1e6)),
+            "config": workload_config(w, args),
+            "parallelism": f"heads x{world} (all-gather of O in the step)" if plan is not None else f"replicas x{world}",
+            "l2": "no flush: Q/K/V/O = %.0f MB > 126 MB L2" % (4 * w.heads * w.tokens * w.d * 2 / 1e6),
             "ms_per_call": ms,
             "effective_flop_per_call": eff_flop, "visited_flop_per_call": vis_flop, "executed_flop_per_call": exe_flop,
             "visited_tflops": vis_flop / (ms * 1e-3) / 1e12,

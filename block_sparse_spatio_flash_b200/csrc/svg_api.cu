@@ -196,13 +196,16 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
                   int d, float scale, const uint8_t* h_route, const void* ws_sp, const void* ws_tm,
                   const svg_geom* geom, const svg_mask* mask, int bq, int bk, int mode, bool dense,
                   void* scratch, size_t scratch_bytes, int32_t* d_status, cudaStream_t st, bool fused = false,
-                  bool qk8 = false) {
+                  bool qk8 = false, bool stall = false) {
   int rc = check_qkvo(q, k, v, o, lse, heads, tokens, d);
   if (rc) return rc;
   if (!scratch || scratch_bytes < kScratchBytes || !aligned(scratch, 16)) return SVG_ERR_ARG;
   if (d_status && !aligned(d_status, 4)) return SVG_ERR_ARG;
   if (bk != 64 && bk != 128) return SVG_ERR_UNSUPPORTED;
   if (qk8 && (d != 128 || fused)) return SVG_ERR_UNSUPPORTED;  // e4m3 QK^T: d = 128, permuted order
+  // fused order gathers rows of a [heads * tokens, d] view whose row coordinate is a signed 32-bit
+  // TMA coordinate
+  if (fused && (int64_t)heads * tokens > (int64_t)INT32_MAX) return SVG_ERR_UNSUPPORTED;
   int num_sms = 0;
   rc = device_info(&num_sms);
   if (rc) return rc;
@@ -229,10 +232,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   P.naive = mode == SVG_MODE_NAIVE ? 1 : 0;
   P.fused = fused && !dense ? 1 : 0;
   P.qk8 = qk8 ? 1 : 0;
-  {  // test hook, read on every call: SVG_TEST_STALL=1 makes the launch time out on purpose
-    const char* ts = getenv("SVG_TEST_STALL");
-    P.inject_stall = (ts && ts[0] == '1' && !pair && !pair1) ? 1 : 0;
-  }
+  P.inject_stall = (stall && !pair && !pair1) ? 1 : 0;  // only svg_test_attention_fwd_stall sets it
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
   P.status = d_status ? d_status : static_cast<int*>(scratch);
@@ -310,31 +310,22 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
 // ---------------------------------------------------------------------------------------
 // Scratch of svg_attention_fwd_noalloc: a file-scope device array, so that callers that
 // cannot allocate need not pass one. In host code `g_noalloc_scratch` only names the
-// symbol; its device address comes from cudaGetSymbolAddress, looked up once per device
-// (with that device current) on the first call there.
+// symbol; its device address comes from cudaGetSymbolAddress on every call, with the
+// caller's device current.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SVG_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
 void* noalloc_scratch(int* rc) {
-  static std::mutex mu;
-  static void* addr[kMaxDevices] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    *rc = SVG_ERR_CUDA;
+  // looked up on every call (cheap, no device work), so that the address always belongs to the
+  // context that is current now, also after a cudaDeviceReset
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) {
+    *rc = record_cuda_error("cudaGetSymbolAddress", e);
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) {
-      *rc = record_cuda_error("cudaGetSymbolAddress", e);
-      return nullptr;
-    }
-    addr[dev] = p;
-  }
-  return addr[dev];
+  return p;
 }
 
 }  // namespace
@@ -465,6 +456,16 @@ int svg_attention_fwd_fused(const void* q, const void* k, const void* v, void* o
   return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
                        tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
                        static_cast<cudaStream_t>(stream), true);
+}
+
+int svg_test_attention_fwd_stall(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,
+                                 int64_t tokens, int32_t d, float scale, const uint8_t* h_route,
+                                 const void* d_ws_spatial, const void* d_ws_temporal, svg_geom geom, svg_mask mask,
+                                 svg_tile tile, int32_t mode, void* d_scratch, size_t scratch_bytes,
+                                 int32_t* d_status, void* stream) {
+  return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
+                       tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
+                       static_cast<cudaStream_t>(stream), false, false, true);
 }
 
 int svg_attention_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, float* lse, int32_t heads,

@@ -85,6 +85,8 @@ _sig = {
                                                _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
     "svg_attention_fwd_qk8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp,
                                              _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
+    "svg_test_attention_fwd_stall": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p,
+                                                    _vp, _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
     "svg_attention_host_buffer_bytes": (_sz, [_i64, _i32, _i32]),
     "svg_attention_fwd_host": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp, _vp,
                                               svg_geom, svg_mask, svg_tile, _i32, _i32, _vp, _sz]),
@@ -216,6 +218,19 @@ def svg_attention_fwd_qk8(q8, k8, v, o, routes, ws_spatial, ws_temporal, geom, m
                                       _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile, mode,
                                       _ptr(scratch), scratch.numel() * scratch.element_size(), _ptr(status),
                                       _stream(stream)), "svg_attention_fwd_qk8")
+    return o
+
+
+def svg_test_attention_fwd_stall(q, k, v, o, routes, ws_spatial, ws_temporal, geom, mask, tile,
+                                 mode=SVG_MODE_SPLIT, scratch=None, lse=None, scale: float = 0.0, status=None,
+                                 stream=None) -> torch.Tensor:
+    """Test hook: svg_attention_fwd whose launch waits on a barrier nothing completes and ends with
+    SVG_ERR_TIMEOUT in its status word after the wait limit."""
+    heads, tokens, d = q.shape
+    _check(_lib.svg_test_attention_fwd_stall(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), heads, tokens, d, scale,
+                                             _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile,
+                                             mode, _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                             _ptr(status), _stream(stream)), "svg_test_attention_fwd_stall")
     return o
 
 

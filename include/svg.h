@@ -39,12 +39,13 @@
  *     built for other parameters) are written to the status word (see svg_read_status).
  *   - Requires a compute capability 10.0 device (B200, sm_100a); otherwise
  *     SVG_ERR_UNSUPPORTED.
- *   - Environment (read by the host code): SVG_KERNEL=pair or SVG_KERNEL=pair1 (read once per
- *     process) makes d = 128 attention run on the two-SM kernels instead of the one-SM kernel,
- *     and SVG_KERNEL=ps makes the one-SM kernel stage P in shared memory instead of tensor
- *     memory, each with the same results up to rounding; SVG_TEST_STALL=1 (read on every call) is a test hook
- *     that makes an attention launch wait on a barrier nothing completes, so that it ends with
- *     SVG_ERR_TIMEOUT in its status word after the wait limit (2 s).
+ *   - Environment (read once per process by the host code): SVG_KERNEL=pair or SVG_KERNEL=pair1
+ *     makes d = 128 attention run on the two-SM kernels instead of the one-SM kernel, and
+ *     SVG_KERNEL=ps makes the one-SM kernel stage P in shared memory instead of tensor memory,
+ *     each with the same results up to rounding.
+ *   - Per-device state (the streams of svg_attention_fwd_host, device attributes) is created on
+ *     first use and belongs to the device's primary context: do not reset a device
+ *     (cudaDeviceReset) while the library is in use on it.
  */
 #ifndef SVG_H_
 #define SVG_H_
@@ -214,8 +215,9 @@ int svg_dense_attention_fwd(const void *q, const void *k, const void *v, void *o
  * SVG_NOALLOC_SCRATCH_BYTES bytes inside the library (every device that loads the library
  * holds it until the process exits). Arguments are those of svg_attention_fwd without
  * d_scratch / scratch_bytes.
- *   - The first call on each device looks up the array's device address (with that device
- *     current); make that first call before any stream capture.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress, with the caller's
+ *     device current); the first lookup on a device may load the library's device code there,
+ *     so make the first call on each device before any stream capture.
  *   - Every call on a device shares the one array and clears it on `stream` before its
  *     kernel runs; calls that overlap on the GPU (other streams, other host threads) race on
  *     it and must be serialised by the caller.
@@ -294,6 +296,8 @@ int svg_attention_fwd_host(const void *h_q, const void *h_k, const void *h_v, vo
  * write each O row back to its original index, so the arithmetic, tile by tile, is that of
  * svg_permute + svg_attention_fwd + svg_permute(inverse) and the results are bitwise equal.
  * Arguments as svg_attention_fwd; lse (nullable) is [heads, tokens] in original order.
+ * SVG_ERR_UNSUPPORTED when heads * tokens exceeds 2^31 - 1 (rows are gathered through a
+ * [heads * tokens, d] view whose row coordinate is a signed 32-bit number).
  */
 int svg_attention_fwd_fused(const void *q, const void *k, const void *v, void *o, float *lse,
                             int32_t heads, int64_t tokens, int32_t d, float scale,
@@ -301,6 +305,20 @@ int svg_attention_fwd_fused(const void *q, const void *k, const void *v, void *o
                             const void *d_ws_temporal, svg_geom geom, svg_mask mask,
                             svg_tile tile, int32_t mode, void *d_scratch, size_t scratch_bytes,
                             int32_t *d_status, void *stream);
+
+/*
+ * Test hook, not a counterpart of anything on the pages: svg_attention_fwd whose softmax warps
+ * first wait on a barrier that nothing completes. That wait gives up after its limit (2 s); the
+ * launch then drains its copies and MMAs, frees its tensor memory, returns early and leaves
+ * SVG_ERR_TIMEOUT in the status word. It lets the failure path run on a GPU without a fault.
+ * Arguments and argument errors as svg_attention_fwd.
+ */
+int svg_test_attention_fwd_stall(const void *q, const void *k, const void *v, void *o, float *lse,
+                                 int32_t heads, int64_t tokens, int32_t d, float scale,
+                                 const uint8_t *h_route, const void *d_ws_spatial,
+                                 const void *d_ws_temporal, svg_geom geom, svg_mask mask,
+                                 svg_tile tile, int32_t mode, void *d_scratch, size_t scratch_bytes,
+                                 int32_t *d_status, void *stream);
 
 /* Reads the device status word of a scratch buffer (or d_status). Synchronises `stream`. */
 int svg_read_status(const void *d_scratch_or_status, int32_t *h_status, void *stream);

@@ -45,8 +45,10 @@ def build_maps(w, g, m, t, routes):
     return maps
 
 
-def run_path(w: syn.Workload, q, k, v, *, mode=0, variant=None, bq=None, bk=None, dense=False, lse=True):
-    """Returns (O [H, N, d] bf16 CPU in original order, LSE [H, N] fp32 CPU in POSITION order, status)."""
+def run_path(w: syn.Workload, q, k, v, *, mode=0, variant=None, bq=None, bk=None, dense=False, lse=True,
+             stall=False):
+    """Returns (O [H, N, d] bf16 CPU in original order, LSE [H, N] fp32 CPU in POSITION order, status).
+    stall: run the launch through the test hook whose wait runs out (svg_test_attention_fwd_stall)."""
     S = svg()
     dev = torch.device("cuda")
     g, m, t = geom_mask_tile(w, variant, bq, bk)
@@ -65,7 +67,8 @@ def run_path(w: syn.Workload, q, k, v, *, mode=0, variant=None, bq=None, bk=None
         S.svg_dense_attention_fwd(qp, kp, vp, o, bk=t.bk, scratch=scratch, lse=ls)
     else:
         maps = build_maps(w, g, m, t, routes)
-        S.svg_attention_fwd(qp, kp, vp, o, routes, maps[0], maps[1], g, m, t, mode=mode, scratch=scratch, lse=ls)
+        fwd = S.svg_test_attention_fwd_stall if stall else S.svg_attention_fwd
+        fwd(qp, kp, vp, o, routes, maps[0], maps[1], g, m, t, mode=mode, scratch=scratch, lse=ls)
     status = S.svg_read_status(scratch)
     if not dense and any(routes):
         out = torch.empty_like(o)
@@ -101,15 +104,33 @@ def oracle_rows(w, q, k, v, h, rows, *, variant=None, bq=None, bk=None, all_kept
                                  **kw)
 
 
-def compare_rows(w, q, k, v, out, lse, rows_per_head=None, **kw):
-    """Check every head on its sampled rows; returns a list of per-head stats."""
+def oracle_rows_cached(cache, key, w, q, k, v, h, rows, **kw):
+    """oracle_rows through a per-row memo: `key` names the inputs and the mask (the same key must
+    mean the same q / k / v and the same mask), so that checks of one workload under several tile
+    shapes of the exact mask share the oracle's rows."""
+    store = cache.setdefault(tuple(key) + (h,), {})
+    missing = np.array([r for r in rows.tolist() if r not in store], dtype=np.int64)
+    if len(missing):
+        o, l = oracle_rows(w, q, k, v, h, missing, **kw)
+        for i, r in enumerate(missing.tolist()):
+            store[r] = (o[i], l[i])
+    return (np.stack([store[r][0] for r in rows.tolist()]),
+            np.array([store[r][1] for r in rows.tolist()], dtype=np.float64))
+
+
+def compare_rows(w, q, k, v, out, lse, rows_per_head=None, cache=None, cache_key=None, **kw):
+    """Check every head on its sampled rows; returns a list of per-head stats. With `cache` (a dict)
+    and `cache_key`, oracle rows are memoised across calls (see oracle_rows_cached)."""
     # LSE rows are in each head's token order, except on the dense path (never permuted)
     permuted = not kw.get("all_kept", False)
     stats = []
     for h in range(w.heads):
         rows = syn.sample_rows(w, h) if rows_per_head is None else rows_per_head(h)
         rows = np.asarray(rows, dtype=np.int64)
-        ref, ref_lse = oracle_rows(w, q, k, v, h, rows, **kw)
+        if cache is not None:
+            ref, ref_lse = oracle_rows_cached(cache, cache_key, w, q, k, v, h, rows, **kw)
+        else:
+            ref, ref_lse = oracle_rows(w, q, k, v, h, rows, **kw)
         got = out[h, torch.as_tensor(rows)].to(torch.float64).numpy()
         diff = got - ref
         rel = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-30))

@@ -183,3 +183,27 @@ def test_qk8_argument_checks(svg):
     p = ctypes.c_void_p(1 << 20)
     assert f(p, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -2   # d = 64
     assert f(None, p, p, p, None, 2, 512, 128, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -1  # null q8
+
+
+def test_fused_rejects_more_rows_than_a_tma_coordinate_holds(svg):
+    """The fused-order call gathers rows of a [heads * tokens, d] view with signed 32-bit row
+    coordinates: heads * tokens above 2^31 - 1 is rejected before any device work."""
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    f = lib.svg_attention_fwd_fused
+    f.argtypes = svg._sig["svg_attention_fwd_fused"][1]
+    g, m, t = svg.make_geom(32, 256, 256), svg.make_mask(1, 16), svg.make_tile(128, 128)
+    tokens = 32 * 256 * 256  # 2^21
+    p = ctypes.c_void_p(1 << 20)
+    routes = (ctypes.c_uint8 * 1024)(*([1] * 1024))
+    assert f(p, p, p, p, None, 1024, tokens, 128, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -2
+
+
+def test_stall_test_entry_checks_arguments_like_the_regular_call(svg):
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    f = lib.svg_test_attention_fwd_stall
+    f.argtypes = svg._sig["svg_test_attention_fwd_stall"][1]
+    g, m, t = svg.make_geom(4, 8, 16), svg.make_mask(1, 16), svg.make_tile(64, 64)
+    routes = (ctypes.c_uint8 * 2)(0, 1)
+    p = ctypes.c_void_p(1 << 20)
+    assert f(None, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -1
+    assert f(p, p, p, p, None, 2, 512, 96, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -2

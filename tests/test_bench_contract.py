@@ -1,6 +1,6 @@
 """Host-side parts of bench.py's JSON contract (CPU): the captured DRAM traffic is reported only for
 the kernel sources, workload and launch shape it was captured on, and both arms print the same
-`config` object apart from how the work is spread."""
+`config` object."""
 import argparse
 
 import bench
@@ -36,12 +36,29 @@ def test_traffic_only_for_the_captured_kernel_and_workload(monkeypatch):
     assert bench.captured_traffic(w, _args()) is None
 
 
-def test_both_arms_share_the_config_keys():
+def test_both_arms_print_the_same_config():
     w = syn.SPATIAL_75K
-    a = bench.workload_config(w, _args(), "replicas x1", "no flush")
-    b = bench.workload_config(w, _args(), "oracle on the host cores of rank 0 of 1", "n/a (host memory)")
-    assert a.keys() == b.keys()
-    assert {k: v for k, v in a.items() if k not in ("parallelism", "l2")} == \
-        {k: v for k, v in b.items() if k not in ("parallelism", "l2")}
+    a = bench.workload_config(w, _args())
+    b = bench.workload_config(w, _args())
+    assert a == b
+    assert "parallelism" not in a and "l2" not in a
     assert a["workload"] == "spatial_75600" and a["tokens"] == 75600 and a["heads"] == 10
     assert a["routes"] == "S" * 10 and a["bq"] == 128 and a["bk"] == 128
+
+
+def test_reference_arm_line_carries_the_workload_config(capsys):
+    """The reference arm's JSON line (rank 0, a tiny bounded sample) prints the same config object as
+    the GPU arm builds for that workload, with the spread of the work outside it."""
+    import json
+    args = argparse.Namespace(steps=1, warmup=3, ref_rows=4, bq=64, bk=64, mode="split")
+    assert bench.run_reference(args, syn.TINY, 1, 0) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"] == bench.workload_config(syn.TINY, args)
+    assert "parallelism" in line and "parallelism" not in line["config"]
+
+
+def test_clock_sampler_writes_outside_the_repository(tmp_path):
+    c = bench.ClockSampler(0)
+    assert not c.path.startswith(bench.ROOT)
+    c2 = bench.ClockSampler(0, str(tmp_path))
+    assert c2.path.startswith(str(tmp_path))

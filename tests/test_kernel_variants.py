@@ -1,7 +1,8 @@
 """The selectable kernels (SVG_KERNEL=pair: 512-row items, two halves per SM; SVG_KERNEL=pair1:
 one 128-row half per SM, key tiles alternating between two softmax groups; SVG_KERNEL=ps: the
-single-SM kernel with P staged in shared memory) against the oracle.
-The kernel choice is read once per process, so each runs in a child process."""
+single-SM kernel with P staged in shared memory) against the oracle, on every entry the option
+reaches: sparse (both modes, both masks), dense, d = 64, fused token order, and for ps the e4m3 QK^T
+call and the bounded-wait path. The kernel choice is read once per process, so each runs in a child process."""
 import os
 import subprocess
 import sys
@@ -15,6 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CHILD = r"""
 import sys
 sys.path.insert(0, {root!r})
+import torch
 from block_sparse_spatio_flash_b200 import synthetic as syn
 from tests import gpu_path as gp
 cases = [
@@ -37,6 +39,31 @@ for w, kw in cases:
     out, lse, st = gp.run_path(w, q, k, v, dense=True, bk=kw.get("bk", 128))
     assert st == 0, st
     gp.compare_rows(w, q, k, v, out, lse, all_kept=True)
+# every other entry the option reaches: d = 64, fused token order, e4m3 QK^T, the bounded-wait path
+w64 = syn.Workload("d64_ragged", frames=5, grid_h=6, grid_w=9, routes=(1, 1, 0), d=64, frame_window=0,
+                   spatial_band=2, bq=64, bk=64)
+for bk in (64, 128):
+    q, k, v = syn.make_qkv(w64, seed_offset=47)
+    out, lse, st = gp.run_path(w64, q, k, v, bk=bk)
+    assert st == 0, st
+    gp.compare_rows(w64, q, k, v, out, lse, bk=bk)
+wf = cases[0][0]
+q, k, v = syn.make_qkv(wf, seed_offset=53)
+want, _, st = gp.run_path(wf, q, k, v, lse=False)
+got, _, st2 = gp.run_fused(wf, q, k, v, lse=False)
+assert st == 0 and st2 == 0, (st, st2)
+assert (got.view(torch.int16) == want.view(torch.int16)).all()
+gp.compare_rows(wf, q, k, v, got, None)
+if {one_sm}:  # the two-SM options leave the e4m3 call and the stall hook to the one-SM kernel
+    q8, k8 = gp.quantize_e4m3(q), gp.quantize_e4m3(k)
+    out, st = gp.run_qk8(wf, q8, k8, v)
+    assert st == 0, st
+    gp.compare_rows(wf, q8, k8, v, out, None)
+    _, _, st = gp.run_path(wf, q, k, v, stall=True)
+    assert st == -4, st
+    out, lse, st = gp.run_path(wf, q, k, v)
+    assert st == 0, st
+    gp.compare_rows(wf, q, k, v, out, lse)
 print("ok")
 """
 
@@ -44,6 +71,7 @@ print("ok")
 @pytest.mark.parametrize("kernel", ["pair", "pair1", "ps"])
 def test_two_sm_kernels_match_oracle(kernel):
     env = dict(os.environ, SVG_KERNEL=kernel)
-    r = subprocess.run([sys.executable, "-c", CHILD.format(root=ROOT)], env=env, cwd=ROOT, capture_output=True,
+    child = CHILD.format(root=ROOT, one_sm=kernel == "ps")
+    r = subprocess.run([sys.executable, "-c", child], env=env, cwd=ROOT, capture_output=True,
                        text=True, timeout=600)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), (r.stdout[-2000:], r.stderr[-4000:])

@@ -1,6 +1,7 @@
 """Head sharding across ranks: the partition, the all-gather of O (gloo ranks on CPU, world sizes
 2 and 3), the pairing of each rank's heads with their own routes (against the oracle), and on one
-GPU the sharded compute of a two-rank plan run rank by rank against the single call."""
+GPU the sharded compute of a two-rank plan, run rank by rank (against the single call and the
+oracle) and as two processes whose device outputs are gathered (against the oracle)."""
 import os
 import socket
 
@@ -176,3 +177,67 @@ def test_sharded_compute_matches_single_call_gpu():
     assert S.svg_read_status(sc) == 0
     got = shard.assemble(blocks, p, torch.empty_like(o_full))
     assert torch.equal(got, o_full)  # same kernel, same rows: bitwise
+    # and the sharded result against the oracle, every row of every head (original order)
+    o_orig = torch.empty_like(got)
+    S.svg_permute(got, o_orig, routes, g, m, inverse=True)
+    torch.cuda.synchronize()
+    q0, k0, v0 = syn.make_qkv(w, seed_offset=17)
+    gp.compare_rows(w, q0, k0, v0, o_orig.cpu(), None)
+
+
+# ------------------------------------------------------------------ GPU: two ranks, device outputs gathered
+GPU_SHARD_W = syn.Workload("shard_gpu_1200", frames=5, grid_h=12, grid_w=20, routes=(1, 0, 1, 1, 0), d=128,
+                           frame_window=1, spatial_band=20)
+
+
+def _gpu_rank_worker(rank, world, port, out):
+    """One rank of a two-process group on the one GPU here: its heads' attention on the device, O back
+    to the original order on the device, then the all-gather of O (gloo, host copies of the device
+    blocks). The ranks' kernels never wait on each other."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from block_sparse_spatio_flash_b200 import svg as S
+        from tests import gpu_path as gp
+        torch.cuda.set_device(0)
+        dev = torch.device("cuda", 0)
+        w = GPU_SHARD_W
+        routes = list(w.routes)
+        g, m, t = gp.geom_mask_tile(w)
+        maps = gp.build_maps(w, g, m, t, routes)
+        summ = [S.svg_tilemap_summary(x) if x is not None else None for x in maps]
+        p = shard.plan_heads(shard.head_costs(routes, summ), world)
+        lr = shard.local_routes(p, rank, routes)
+        q, k, v = syn.make_qkv(w, seed_offset=29)
+        ql, kl, vl = (shard.local_heads(x, p, rank).to(dev) for x in (q, k, v))
+        qp, kp, vp = (torch.empty_like(x) for x in (ql, kl, vl))
+        for a, b in ((ql, qp), (kl, kp), (vl, vp)):
+            S.svg_permute(a, b, lr, g, m)
+        o = torch.empty_like(qp)
+        sc = S.alloc_scratch(dev)
+        shard.attention_fwd_local(qp, kp, vp, o, p, rank, routes, maps[0], maps[1], g, m, t, scratch=sc)
+        o_orig = torch.empty_like(o)
+        S.svg_permute(o, o_orig, lr, g, m, inverse=True)
+        torch.cuda.synchronize()
+        status = S.svg_read_status(sc)
+        full = shard.gather_heads(o_orig.cpu(), p)
+        ok = status == 0 and tuple(full.shape) == (w.heads, w.tokens, w.d)
+        if ok and rank == 0:
+            gp.compare_rows(w, q, k, v, full, None)
+        out[rank] = bool(ok)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_sharded_ranks_gather_device_outputs_gpu():
+    from block_sparse_spatio_flash_b200 import build
+    build.build()
+    world = 2
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as man:
+        out = man.dict()
+        mp.spawn(_gpu_rank_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res == {0: True, 1: True}

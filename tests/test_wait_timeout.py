@@ -1,5 +1,5 @@
 """Failure detection on the GPU without a fault: a launch whose softmax warps wait on a barrier that
-nothing completes (test hook SVG_TEST_STALL=1) must give up after the bounded wait, report
+nothing completes (the test entry point svg_test_attention_fwd_stall) must give up after the bounded wait, report
 SVG_ERR_TIMEOUT through the status word, drain its copies and MMAs, free TMEM and return; the next
 launch in the same context must then run normally and match the oracle."""
 import pytest
@@ -20,12 +20,10 @@ def S():
     return gp.svg()
 
 
-def test_stalled_wait_reports_timeout_and_context_survives(S, monkeypatch):
+def test_stalled_wait_reports_timeout_and_context_survives(S):
     q, k, v = syn.make_qkv(W, seed_offset=31)
-    monkeypatch.setenv("SVG_TEST_STALL", "1")
-    _, _, st = gp.run_path(W, q, k, v)
+    _, _, st = gp.run_path(W, q, k, v, stall=True)
     assert st == S.SVG_ERR_TIMEOUT
-    monkeypatch.delenv("SVG_TEST_STALL")
     out, lse, st = gp.run_path(W, q, k, v)
     assert st == 0
     gp.compare_rows(W, q, k, v, out, lse)

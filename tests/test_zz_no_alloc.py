@@ -57,16 +57,26 @@ def test_noalloc_matches_regular_entry_point_twice():
     assert S.svg_read_status(scratch) == 0
 
     status = torch.full((1,), 12345, dtype=torch.int32, device=dev)
+    outs = [torch.full_like(qp, float("nan")) for _ in range(3)]
+    lses = [torch.full_like(ref_lse, float("nan")) for _ in range(3)]
     for call in range(2):
-        o = torch.full_like(qp, float("nan"))
-        lse = torch.full_like(ref_lse, float("nan"))
+        o, lse = outs[call], lses[call]
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         S.svg_attention_fwd_noalloc(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, lse=lse, status=status)
         torch.cuda.synchronize()
+        if call == 1:  # the library is loaded and its array resident: a call allocates no device memory
+            assert torch.cuda.mem_get_info()[0] == free_before
         assert int(status.item()) == 0, f"call {call}: device status {int(status.item())}"
         ok, rel, mx = _close(o.float(), ref.float())
         assert ok, (call, rel, mx)
         assert torch.isfinite(o.float()).all()
         assert float((lse - ref_lse).abs().max()) <= 5e-3
+    # without a status pointer the status word inside the library's own array is used
+    S.svg_attention_fwd_noalloc(qp, kp, vp, outs[2], routes, ws[0], ws[1], g, m, t, lse=lses[2])
+    torch.cuda.synchronize()
+    ok, rel, mx = _close(outs[2].float(), ref.float())
+    assert ok, ("no status pointer", rel, mx)
 
 
 def test_noalloc_rejects_bad_arguments_without_touching_the_device():
