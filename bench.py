@@ -478,6 +478,7 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
     work = torch.empty(S.svg_route_work_bytes(w.heads, w.tokens, w.d, rows.numel()), dtype=torch.uint8, device=dev)
     out["route_ms"] = time_events(lambda: S.svg_route_heads(q, k, v, g, m, rows, rt, work=work), 5, stream)
     out["route_rows_per_head"] = int(rows.numel())
+    out["scheduler"] = scheduler_compare(S, w, qp, kp, vp, o, routes, ws, g, m, t, scratch, stream, dev)
     out["workloads"] = other_workloads(S, P, stream, dev)
     out["tile_sweep_mixed_75600"] = tile_sweep(S, stream, dev)
     st = S.svg_read_status(scratch)
@@ -523,6 +524,39 @@ def tile_sweep(S, stream, dev):
     return res
 
 
+def trace_stats(tr):
+    """Balance of one traced launch from its per-CTA records (start ns, end ns, items, half-tiles):
+    span of the launch, busy time per CTA (start to end of the CTA), the tail (last CTA end minus the
+    median CTA end) and the spread of the work the CTAs took."""
+    t = tr[tr[:, 0] > 0].to(torch.float64)
+    if t.numel() == 0:
+        return None
+    start, end = t[:, 0], t[:, 1]
+    busy = (end - start) / 1e6
+    span = float(end.max() - start.min()) / 1e6
+    return {"ctas": int(t.shape[0]), "span_ms": span, "busy_max_ms": float(busy.max()),
+            "busy_mean_ms": float(busy.mean()), "busy_min_ms": float(busy.min()),
+            "tail_ms": float(end.max() - end.median()) / 1e6,
+            "idle_frac": 1.0 - float(busy.sum()) / (t.shape[0] * span) if span > 0 else 0.0,
+            "tiles_max": int(t[:, 3].max()), "tiles_mean": float(t[:, 3].mean()), "tiles_min": int(t[:, 3].min()),
+            "items_max": int(t[:, 2].max()), "items_min": int(t[:, 2].min())}
+
+
+def scheduler_compare(S, w, qp, kp, vp, o, routes, ws, g, m, t, sc, stream, dev, iters=5):
+    """Both scheduling orders of the persistent kernel on one workload: ms per call (untraced) and the
+    per-CTA balance of one traced call each."""
+    n = torch.cuda.get_device_properties(dev).multi_processor_count
+    tr = torch.zeros((n, 4), dtype=torch.int64, device=dev)
+    out = {}
+    for name, order in (("head_major", S.SVG_ORDER_HEAD_MAJOR), ("work", S.SVG_ORDER_WORK)):
+        ms = time_events(lambda: S.svg_attention_fwd_ex(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, scratch=sc,
+                                                        order=order), iters, stream)
+        S.svg_attention_fwd_ex(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, scratch=sc, order=order, cta_trace=tr)
+        torch.cuda.synchronize()
+        out[name] = {"ms": ms, "trace": trace_stats(tr.cpu())}
+    return out
+
+
 def other_workloads(S, P, stream, dev):
     """Attention time (split mode, permuted inputs, 128 x 128 tiles) of the other workloads of the
     pages' shapes: all-temporal heads at 75,600 tokens (sink-prefix and fully space-major token
@@ -558,6 +592,7 @@ def other_workloads(S, P, stream, dev):
                        "visited_tflops": vis / (ms * 1e-3) / 1e12,
                        "visited_frac_of_peak": vis / (ms * 1e-3) / 1e12 / float(P["bf16_tflops"]),
                        "fused_order_ms": ms_fused, "permuted_path_ms": ms + 4 * ms_perm,
+                       "scheduler": scheduler_compare(S, w, qp, kp, vp, o, routes, ws, g, m, t, sc, stream, dev),
                        "status": S.svg_read_status(sc)}
         del q, k, v, qp, kp, vp, o, ws
         torch.cuda.empty_cache()

@@ -2,8 +2,10 @@
 
     python -m block_sparse_spatio_flash_b200.build [--verbose]
 
-Produces block_sparse_spatio_flash_b200/lib/libsvgattn.so. The library links the CUDA
-runtime statically and depends on no torch symbol; nvcc cross-compiles it on a machine
+Produces block_sparse_spatio_flash_b200/lib/libsvgattn.so and, with build(checked=True), the
+checked build lib/libsvgattn_checked.so (-DSVG_CHECKED=1: device-side bounds checks that count
+failures instead of trapping; loaded when SVG_CHECKED=1 is set, see svg.py). The libraries link the
+CUDA runtime statically and depend on no torch symbol; nvcc cross-compiles them on a machine
 without a GPU.
 """
 from __future__ import annotations
@@ -18,7 +20,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libsvgattn.so")
-SOURCES = ["svg_api.cu", "svg_tilemap.cu", "svg_permute.cu", "svg_attention.cu", "svg_attention2.cu", "svg_attention3.cu", "svg_route.cu"]
+LIB_CHECKED = os.path.join(LIBDIR, "libsvgattn_checked.so")
+SOURCES = ["svg_api.cu", "svg_tilemap.cu", "svg_permute.cu", "svg_attention.cu", "svg_route.cu"]
 HEADERS = ["svg_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -30,27 +33,30 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", "svg.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not _stale(lib):
+        return lib
     os.makedirs(LIBDIR, exist_ok=True)
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp"]
+           "-I", os.path.join(ROOT, "include"), "-o", lib + ".tmp"]
+    if checked:
+        cmd += ["-DSVG_CHECKED=1"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="--verbose" in sys.argv))
+    print(build(force=True, verbose="--verbose" in sys.argv, checked="--checked" in sys.argv))

@@ -16,8 +16,6 @@ int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* 
 int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const uint8_t* h_route, svg_geom geom,
                    svg_mask mask, int inverse, int num_sms, cudaStream_t st);
 int launch_attention(const AttnParams& P, int d, int bk, int grid, bool p_smem, cudaStream_t st);
-int launch_attention_pair(const AttnParams& P, int bk, int max_clusters, cudaStream_t st);
-int launch_attention_pair1(const AttnParams& P, int bk, cudaStream_t st);
 size_t route_work_bytes(int heads, int64_t N, int d, int n_rows);
 int launch_route(const void* q, const void* k, const void* v, int heads, int N, int d, float scale, svg_geom geom,
                  svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
@@ -28,6 +26,20 @@ using namespace svg;
 
 namespace svg {
 int record_cuda_error(const char* what, int cuda_error);
+unsigned int* checks_counter();
+}
+
+// Failed-check counter of the checked build (see SVG_CHECKED in svg_common.cuh).
+static __device__ unsigned int g_checks_failed;
+
+// Device address of the counter (null in the release build, whose kernels never use it).
+unsigned int* svg::checks_counter() {
+#if SVG_CHECKED
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_checks_failed) == cudaSuccess ? static_cast<unsigned int*>(p) : nullptr;
+#else
+  return nullptr;
+#endif
 }
 
 namespace {
@@ -152,24 +164,24 @@ int encode_rows_map(CUtensorMap* m, const void* base, int heads, int64_t tokens,
   return SVG_OK;
 }
 
-// The single-SM kernel serves every call; SVG_KERNEL=pair in the environment (read once)
-// selects the SM-pair kernel (two-SM MMAs, each SM loading half of every K/V tile) for d = 128,
-// to compare the two.
-bool use_pair_kernel(int d) {
-  static const bool pair = [] {
-    const char* v = getenv("SVG_KERNEL");
-    return v && strcmp(v, "pair") == 0;
-  }();
-  return d == 128 && pair;
-}
-
-// SVG_KERNEL=pair1: SM pairs with one 128-row half per SM and double-buffered scores (d = 128).
-bool use_pair1_kernel(int d) {
-  static const bool pair1 = [] {
-    const char* v = getenv("SVG_KERNEL");
-    return v && strcmp(v, "pair1") == 0;
-  }();
-  return d == 128 && pair1;
+// [heads, T, S, d] bf16 (original frame-major order) viewed as a 4-D tensor (d, patch, frame, head);
+// box = 64 columns x 1 patch x run_len frames x 1 head: one patch's run of frames, rows S apart in
+// memory, lands as run_len consecutive 128-byte rows.
+int encode_run_map(CUtensorMap* m, const void* base, int heads, int frames, int patches, int d, int run_len) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return record_cuda_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", (int)cudaErrorSymbolNotFound);
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)patches, (cuuint64_t)frames, (cuuint64_t)heads};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)patches * d * 2, (cuuint64_t)frames * patches * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)run_len, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (runs): CUresult %d", (int)r);
+    return SVG_ERR_CUDA;
+  }
+  return SVG_OK;
 }
 
 // SVG_KERNEL=ps: the single-SM kernel with P staged in shared memory, so that the next key tile's
@@ -196,11 +208,14 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
                   int d, float scale, const uint8_t* h_route, const void* ws_sp, const void* ws_tm,
                   const svg_geom* geom, const svg_mask* mask, int bq, int bk, int mode, bool dense,
                   void* scratch, size_t scratch_bytes, int32_t* d_status, cudaStream_t st, bool fused = false,
-                  bool qk8 = false, bool stall = false) {
+                  bool qk8 = false, bool stall = false, int order = kOrderHeadMajor,
+                  unsigned long long* cta_trace = nullptr, int trace_ctas = 0) {
   int rc = check_qkvo(q, k, v, o, lse, heads, tokens, d);
   if (rc) return rc;
   if (!scratch || scratch_bytes < kScratchBytes || !aligned(scratch, 16)) return SVG_ERR_ARG;
   if (d_status && !aligned(d_status, 4)) return SVG_ERR_ARG;
+  if (order != kOrderHeadMajor && order != kOrderWork) return SVG_ERR_ARG;
+  if (cta_trace && (trace_ctas < 1 || !aligned(cta_trace, 8))) return SVG_ERR_ARG;
   if (bk != 64 && bk != 128) return SVG_ERR_UNSUPPORTED;
   if (qk8 && (d != 128 || fused)) return SVG_ERR_UNSUPPORTED;  // e4m3 QK^T: d = 128, permuted order
   // fused order gathers rows of a [heads * tokens, d] view whose row coordinate is a signed 32-bit
@@ -215,14 +230,11 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   std::lock_guard<std::mutex> lock(mu);
   memset(&P, 0, sizeof(P));
   const int N = (int)tokens;
-  const bool pair = use_pair_kernel(d) && !fused && !qk8;
-  const bool pair1 = use_pair1_kernel(d) && !fused && !pair && !qk8;
   P.H = heads;
   P.N = N;
   P.nk = (N + bk - 1) / bk;
   P.npairs = (N + kPairRows - 1) / kPairRows;
-  P.nquads = (N + kQuadRows - 1) / kQuadRows;
-  const int64_t items = (int64_t)heads * (pair ? P.nquads : P.npairs);
+  const int64_t items = (int64_t)heads * P.npairs;
   if (items > 0x7FFFFFFF) return SVG_ERR_ARG;
   P.n_items = (int)items;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
@@ -232,11 +244,15 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
   P.naive = mode == SVG_MODE_NAIVE ? 1 : 0;
   P.fused = fused && !dense ? 1 : 0;
   P.qk8 = qk8 ? 1 : 0;
-  P.inject_stall = (stall && !pair && !pair1) ? 1 : 0;  // only svg_test_attention_fwd_stall sets it
+  P.inject_stall = stall ? 1 : 0;  // only svg_test_attention_fwd_stall sets it
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
   P.status = d_status ? d_status : static_cast<int*>(scratch);
+  P.checks = checks_counter();
   P.counter = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(scratch) + 8);
+  P.counter64 = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kCounter64Off);
+  P.cta_trace = cta_trace;
+  P.trace_ctas = cta_trace ? trace_ctas : 0;
   if (!dense) {
     if (!h_route || !geom || !mask) return SVG_ERR_ARG;
     if (!geom_ok(*geom) || !mask_ok(*geom, *mask)) return SVG_ERR_ARG;
@@ -250,7 +266,9 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
       if (h_route[h] > 1) return SVG_ERR_ARG;
       if (h_route[h]) P.route_bits[h >> 5] |= 1u << (h & 31);
       P.uses[h_route[h]] = 1;
+      ++P.hc[h_route[h]];
     }
+    P.order = order;
     for (int c = 0; c < 2; ++c) {
       P.g[c] = make_geom(*geom, *mask, c);
       if (!P.uses[c]) continue;
@@ -262,10 +280,7 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
       P.pair_ent[c] = reinterpret_cast<const uint32_t*>(b + L.pair_ent);
       P.pair_cnt[c] = reinterpret_cast<const uint32_t*>(b + L.pair_cnt);
       P.pair_order[c] = reinterpret_cast<const uint32_t*>(b + L.pair_order);
-      P.quad_ptr[c] = reinterpret_cast<const uint32_t*>(b + L.quad_ptr);
-      P.quad_ent[c] = reinterpret_cast<const uint32_t*>(b + L.quad_ent);
-      P.quad_cnt[c] = reinterpret_cast<const uint32_t*>(b + L.quad_cnt);
-      P.quad_order[c] = reinterpret_cast<const uint32_t*>(b + L.quad_order);
+      P.pair_grp[c] = reinterpret_cast<const uint32_t*>(b + L.pair_grp);
     }
     P.variant = mask->variant;
     P.bq = bq;
@@ -280,26 +295,36 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
     P.exp_bq = bq;
     P.exp_bk = bk;
   }
-  // TMA boxes: Q 128 rows; one-SM kernel K and V bk rows; SM-pair kernel: each SM loads bk/2
-  // keys of K (all 128 dims) and all bk keys of V for 64 of the dims.
+  // TMA boxes: Q 128 rows, K and V bk rows.
   if (qk8) {
     if ((rc = encode_qk8_map(&P.tm_q, q, heads, N, d, 128))) return rc;
     if ((rc = encode_qk8_map(&P.tm_k, k, heads, N, d, bk))) return rc;
   } else {
     if ((rc = encode_qkv_map(&P.tm_q, q, heads, N, d, 128))) return rc;
-    if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, (pair || pair1) ? bk / 2 : bk))) return rc;
+    if ((rc = encode_qkv_map(&P.tm_k, k, heads, N, d, bk))) return rc;
   }
   if ((rc = encode_qkv_map(&P.tm_v, v, heads, N, d, bk))) return rc;
   if (P.fused && P.uses[SVG_ROUTE_TEMPORAL]) {
     if ((rc = encode_rows_map(&P.tm_q2, q, heads, N, d))) return rc;
     if ((rc = encode_rows_map(&P.tm_k2, k, heads, N, d))) return rc;
     if ((rc = encode_rows_map(&P.tm_v2, v, heads, N, d))) return rc;
+    // runs of one patch's frames as boxes: frames [F0, T) after the sink prefix, or all T frames
+    // in the fully space-major order; runs shorter than 4 rows are gathered instead
+    const bool fsm = mask->layout == SVG_LAYOUT_FULL_SPACE_MAJOR;
+    const int run = fsm ? geom->frames : geom->frames - mask->sink_frames;
+    if (run >= 4 && run <= 256) {
+      const int S = geom->grid_h * geom->grid_w;
+      P.run_len = run;
+      P.run_t0 = fsm ? 0 : mask->sink_frames;
+      if ((rc = encode_run_map(&P.tm_q4, q, heads, geom->frames, S, d, run))) return rc;
+      if ((rc = encode_run_map(&P.tm_k4, k, heads, geom->frames, S, d, run))) return rc;
+      if ((rc = encode_run_map(&P.tm_v4, v, heads, geom->frames, S, d, run))) return rc;
+    }
   }
   cudaError_t me = cudaMemsetAsync(scratch, 0, kScratchBytes, st);
   if (me == cudaSuccess && d_status) me = cudaMemsetAsync(d_status, 0, sizeof(int32_t), st);
+  if (me == cudaSuccess && cta_trace) me = cudaMemsetAsync(cta_trace, 0, 32 * (size_t)trace_ctas, st);
   if (me != cudaSuccess) return record_cuda_error("cudaMemsetAsync(scratch)", me);
-  if (pair) return launch_attention_pair(P, bk, (int)(P.n_items < num_sms / 2 ? P.n_items : num_sms / 2), st);
-  if (pair1) return launch_attention_pair1(P, bk, st);
   const int grid = (int)(P.n_items < num_sms ? P.n_items : num_sms);
   return launch_attention(P, d, bk, grid, use_p_smem(), st);
 }
@@ -340,6 +365,25 @@ extern "C" {
 
 const char* svg_last_cuda_error(void) { return g_last_error; }
 
+int svg_checked_build(void) { return SVG_CHECKED ? 1 : 0; }
+
+int svg_checks_failed(uint32_t* h_count, int32_t reset) {
+  if (!h_count) return SVG_ERR_ARG;
+  *h_count = 0;
+#if SVG_CHECKED
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(h_count, g_checks_failed, sizeof(uint32_t));
+  if (e == cudaSuccess && reset) {
+    const uint32_t z = 0;
+    e = cudaMemcpyToSymbol(g_checks_failed, &z, sizeof(uint32_t));
+  }
+  if (e != cudaSuccess) return record_cuda_error("svg_checks_failed", e);
+#else
+  (void)reset;
+#endif
+  return SVG_OK;
+}
+
 int svg_version(void) { return 10000; }
 
 const char* svg_error_string(int code) {
@@ -373,14 +417,10 @@ int svg_tilemap_get_layout(svg_geom geom, svg_tile tile, svg_tilemap_layout* out
   out->pair_ent = L.pair_ent;
   out->pair_cnt = L.pair_cnt;
   out->pair_order = L.pair_order;
-  out->quad_ptr = L.quad_ptr;
-  out->quad_ent = L.quad_ent;
-  out->quad_cnt = L.quad_cnt;
-  out->quad_order = L.quad_order;
+  out->pair_grp = L.pair_grp;
   out->nq = L.nq;
   out->nk = L.nk;
   out->npairs = L.npairs;
-  out->nquads = L.nquads;
   return SVG_OK;
 }
 
@@ -413,8 +453,6 @@ int svg_tilemap_summary(const void* d_ws, svg_tilemap_summary_t* h_out, void* st
   h_out->visited_area = h.visited_area;
   h_out->pair_entries = h.pair_entries;
   h_out->pair_half_tiles = h.pair_half_tiles;
-  h_out->quad_entries = h.quad_entries;
-  h_out->quad_phase_tiles = h.quad_phase_tiles;
   return SVG_OK;
 }
 
@@ -456,6 +494,18 @@ int svg_attention_fwd_fused(const void* q, const void* k, const void* v, void* o
   return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
                        tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
                        static_cast<cudaStream_t>(stream), true);
+}
+
+int svg_attention_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,
+                         int64_t tokens, int32_t d, float scale, const uint8_t* h_route, const void* d_ws_spatial,
+                         const void* d_ws_temporal, svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
+                         void* d_scratch, size_t scratch_bytes, int32_t* d_status, const svg_launch_opts* opts,
+                         void* stream) {
+  if (!opts) return SVG_ERR_ARG;
+  return run_attention(q, k, v, o, lse, heads, tokens, d, scale, h_route, d_ws_spatial, d_ws_temporal, &geom, &mask,
+                       tile.bq, tile.bk, mode, false, d_scratch, scratch_bytes, d_status,
+                       static_cast<cudaStream_t>(stream), false, false, false, opts->order,
+                       reinterpret_cast<unsigned long long*>(opts->d_cta_trace), opts->trace_ctas);
 }
 
 int svg_test_attention_fwd_stall(const void* q, const void* k, const void* v, void* o, float* lse, int32_t heads,

@@ -83,7 +83,7 @@ struct ItemInfo {
 //   2NS + 14       drain         final MMA completion
 //   2NS + 15       never         completed by nothing (test hook: a wait that runs out)
 //   2NS + 16 + h   s_free[h]     (PS) S_h loaded by the softmax, its TMEM columns free (128 arrivals)
-//   2NS + 18 ...   two ItemInfo slots, TMEM base, abort flag, workspace check
+//   2NS + 18 ...   two ItemInfo slots, TMEM base, abort flag, workspace check, trace counts
 template <int NS>
 struct Ctl {
   uint32_t base;  // shared address of the control block
@@ -105,7 +105,8 @@ struct Ctl {
   static constexpr uint32_t kTmemOff = kItemsOff + 96;
   static constexpr uint32_t kAbortOff = kTmemOff + 8;
   static constexpr uint32_t kBadWsOff = kAbortOff + 8;
-  static constexpr uint32_t kBytes = kBadWsOff + 8;
+  static constexpr uint32_t kTraceOff = kBadWsOff + 8;  // items, half-tiles of this CTA (producer)
+  static constexpr uint32_t kBytes = kTraceOff + 8;
 };
 
 __device__ __forceinline__ int ld_shared_volatile(uint32_t addr) {
@@ -196,13 +197,32 @@ __device__ __forceinline__ uint32_t dense_entry(const AttnParams& P, const ItemI
 
 template <int BK>
 __device__ __forceinline__ uint32_t get_entry(const AttnParams& P, const ItemInfo& it, int e) {
-  return P.dense ? dense_entry<BK>(P, it, e) : __ldg(it.ents + e);
+  if (P.dense) return dense_entry<BK>(P, it, e);
+  if (!check_ok(e >= 0 && e < it.count, P.checks)) return 0u;
+  const uint32_t ent = __ldg(it.ents + e);
+  return check_ok(ent_kt(ent) < (uint32_t)P.nk, P.checks) ? ent : (ent & ~0x0FFFFFFFu);
 }
 
 __device__ __forceinline__ int route_of(const AttnParams& P, int h) {
   return (P.route_bits[h >> 5] >> (h & 31)) & 1;
 }
 
+// The item's execution list: pair `pair` of route class it.cls.
+__device__ __forceinline__ void fill_sparse_item(const AttnParams& P, ItemInfo& it) {
+  const int c = it.cls;
+  if (!check_ok((unsigned)it.pair < (unsigned)P.npairs, P.checks)) it.pair = 0;
+  const uint32_t b0 = __ldg(P.pair_ptr[c] + it.pair), b1 = __ldg(P.pair_ptr[c] + it.pair + 1);
+  it.count = (int)(b1 - b0);
+  it.ents = P.pair_ent[c] + b0;
+  it.nA = (int)__ldg(P.pair_cnt[c] + 2 * it.pair);
+  it.nB = (int)__ldg(P.pair_cnt[c] + 2 * it.pair + 1);
+  if (!check_ok(b0 <= b1 && (uint64_t)b1 <= (uint64_t)P.npairs * (uint64_t)P.nk && it.nA <= it.count &&
+                    it.nB <= it.count && it.count <= P.nk,
+                P.checks))
+    it.count = it.nA = it.nB = 0;
+}
+
+// Head-major order: counter value idx -> head idx / npairs, that head's items heaviest first.
 template <int BK>
 __device__ ItemInfo decode_item(const AttnParams& P, uint32_t idx) {
   ItemInfo it;
@@ -219,15 +239,167 @@ __device__ ItemInfo decode_item(const AttnParams& P, uint32_t idx) {
     it.nB = (j * kPairRows + kHalfRows < P.N) ? P.nk : 0;
     it.ents = nullptr;
   } else {
-    const int c = it.cls;
-    it.pair = (int)__ldg(P.pair_order[c] + j);
-    const uint32_t b0 = __ldg(P.pair_ptr[c] + it.pair), b1 = __ldg(P.pair_ptr[c] + it.pair + 1);
-    it.count = (int)(b1 - b0);
-    it.ents = P.pair_ent[c] + b0;
-    it.nA = (int)__ldg(P.pair_cnt[c] + 2 * it.pair);
-    it.nB = (int)__ldg(P.pair_cnt[c] + 2 * it.pair + 1);
+    it.pair = (int)__ldg(P.pair_order[it.cls] + j);
+    fill_sparse_item(P, it);
   }
   return it;
+}
+
+// ---- work-ordered scheduler -------------------------------------------------------------
+// Every head of a route class has the same items with the same work, so the items of a class in
+// descending work, taken head by head within each run of equal work, form the class's sequence;
+// the two classes' sequences are merged by work (ties to the spatial class) through one 64-bit
+// counter holding both positions. This is longest-processing-time-first over all (head, item)
+// pairs, with the heads of one run kept together so that items in flight share K / V rows in L2.
+
+// Work (active 128-row half-tiles) of position p of class c's order.
+__device__ __forceinline__ int work_at(const AttnParams& P, int c, uint32_t p) {
+  const uint32_t g = __ldg(P.pair_order[c] + p);
+  return (int)(__ldg(P.pair_cnt[c] + 2 * g) + __ldg(P.pair_cnt[c] + 2 * g + 1));
+}
+
+// The r-th head (0-based, ascending) whose route is c.
+__device__ int head_of_rank(const AttnParams& P, int c, int r) {
+  const int words = (P.H + 31) >> 5;
+  for (int w = 0; w < words; ++w) {
+    uint32_t bits = c ? P.route_bits[w] : ~P.route_bits[w];
+    if (w == words - 1 && (P.H & 31)) bits &= (1u << (P.H & 31)) - 1u;
+    const int n = __popc(bits);
+    if (r < n) {
+      for (int i = 0; i < r; ++i) bits &= bits - 1u;
+      return w * 32 + __ffs(bits) - 1;
+    }
+    r -= n;
+  }
+  return 0;  // unreachable for r < heads of class c
+}
+
+// Claims the next (class, position) in merged work order; false when both sequences are done.
+// A failed compare-and-swap means another CTA claimed an item, so the retries of one CTA are
+// bounded by the number of items; the cap only guards against a corrupted counter.
+__device__ bool claim_work_item(const AttnParams& P, int& cls, uint32_t& pos) {
+  const uint64_t n0 = (uint64_t)P.hc[0] * (uint64_t)P.npairs, n1 = (uint64_t)P.hc[1] * (uint64_t)P.npairs;
+  unsigned long long cur = atomicAdd(P.counter64, 0ull);
+  for (uint32_t tries = 0; tries < (1u << 28); ++tries) {
+    const uint32_t i0 = (uint32_t)cur, i1 = (uint32_t)(cur >> 32);
+    const int w0 = i0 < n0 ? work_at(P, 0, i0 / (uint32_t)P.hc[0]) : -1;
+    const int w1 = i1 < n1 ? work_at(P, 1, i1 / (uint32_t)P.hc[1]) : -1;
+    if (w0 < 0 && w1 < 0) return false;
+    const int c = w0 >= w1 ? 0 : 1;
+    const unsigned long long nxt = cur + (c ? (1ull << 32) : 1ull);
+    const unsigned long long prev = atomicCAS(P.counter64, cur, nxt);
+    if (prev == cur) {
+      cls = c;
+      pos = c ? i1 : i0;
+      return true;
+    }
+    cur = prev;
+  }
+  atomicCAS(P.status, 0, SVG_ERR_TIMEOUT);
+  return false;
+}
+
+// Position pos of class c's sequence -> (head, item).
+__device__ ItemInfo decode_work_item(const AttnParams& P, int c, uint32_t pos) {
+  ItemInfo it;
+  memset(&it, 0, sizeof(it));
+  const uint32_t hc = (uint32_t)P.hc[c];
+  const uint32_t p = pos / hc;
+  const uint32_t s = __ldg(P.pair_grp[c] + 2 * p), e = __ldg(P.pair_grp[c] + 2 * p + 1);
+  const uint32_t len = e - s, o = pos - hc * s;
+  if (!check_ok(p < (uint32_t)P.npairs && s <= p && p < e && e <= (uint32_t)P.npairs && o < hc * len, P.checks))
+    return it;  // not valid: this CTA stops taking items
+  it.valid = 1;
+  it.cls = c;
+  it.head = head_of_rank(P, c, (int)(o / len));
+  it.pair = (int)__ldg(P.pair_order[c] + s + o % len);
+  fill_sparse_item(P, it);
+  return it;
+}
+
+// ---- fused token order: the rows of a temporal head's tile, read where they lie ------------
+// Positions [p0, p0 + ROWS) of a temporal head's token order go to a ROWS-row tile (64-column chunks
+// ROWS * 128 bytes apart, 128-byte swizzle). Rows of the sink prefix are contiguous in the original
+// order: one tiled copy per chunk. Past the prefix the order runs through one patch's frames at a
+// time (run_len positions whose rows are S apart in the original order): every run lying wholly
+// inside the tile is one 4-D box copy per chunk, and the 4-row groups that hold rows of the partial
+// runs at the tile's edges (or rows past the sequence end, clamped to the last row) are gathered
+// row by row. A gathered group may also hold rows of a whole run; both copies then write the same
+// bytes there. The byte count covers every copy, duplicates included.
+struct FusedPlan {
+  int kind;        // 0: inside the sink prefix, 1: gather every group, 2: runs and edge groups
+  int n_box, u_a;  // whole runs u_a .. u_a + n_box - 1 (patch index = run index)
+  uint32_t gmask;  // 4-row groups to gather (bit = group = lane)
+};
+
+template <int ROWS>
+__device__ __forceinline__ FusedPlan fused_plan(const AttnParams& P, int p0, int lane) {
+  const MaskGeom& g = P.g[SVG_ROUTE_TEMPORAL];
+  const int pre = sink_end(g), R = P.run_len;
+  FusedPlan f;
+  f.n_box = 0;
+  f.u_a = 0;
+  f.gmask = 0;
+  constexpr uint32_t kAll = ROWS / 4 >= 32 ? 0xFFFFFFFFu : ((1u << (ROWS / 4)) - 1u);
+  if (p0 + ROWS <= pre) {
+    f.kind = 0;
+    return f;
+  }
+  if (p0 < pre || R == 0) {
+    f.kind = 1;
+    f.gmask = kAll;
+    return f;
+  }
+  f.kind = 2;
+  const int q0 = p0 - pre;
+  const int u_a = (q0 + R - 1) / R;  // first run that starts inside the tile
+  int u_end = (q0 + ROWS) / R;       // runs [u_a, u_end) end inside the tile
+  const int runs = (g.N - pre) / R;
+  if (u_end > runs) u_end = runs;
+  f.u_a = u_a;
+  f.n_box = u_end > u_a ? u_end - u_a : 0;
+  const int c0 = f.n_box ? u_a * R - q0 : 0, c1 = f.n_box ? u_end * R - q0 : 0;  // rows the boxes cover
+  const int r0 = 4 * lane;
+  const bool need = r0 < ROWS && !(r0 >= c0 && r0 + 4 <= c1);
+  f.gmask = __ballot_sync(0xFFFFFFFFu, need) & kAll;
+  return f;
+}
+
+template <int ROWS, int CHUNKS>
+__device__ __forceinline__ uint32_t fused_bytes(const AttnParams& P, const FusedPlan& f) {
+  if (f.kind == 0) return (uint32_t)(ROWS * 128 * CHUNKS);
+  return ((uint32_t)f.n_box * (uint32_t)P.run_len * 128u + (uint32_t)__popc(f.gmask) * 512u) * CHUNKS;
+}
+
+template <int ROWS, int CHUNKS>
+__device__ __forceinline__ void fused_issue(const AttnParams& P, const FusedPlan& f, const CUtensorMap* tile_map,
+                                            const CUtensorMap* box_map, const CUtensorMap* row_map, uint32_t dst,
+                                            uint32_t bar, int head, int p0, int lane) {
+  if (f.kind == 0) {
+    if (lane == 0)
+      for (int ch = 0; ch < CHUNKS; ++ch) tma_load_3d(dst + ch * (ROWS * 128), tile_map, bar, ch * 64, p0, head);
+    return;
+  }
+  const MaskGeom& g = P.g[SVG_ROUTE_TEMPORAL];
+  if (lane < f.n_box) {
+    const int u = f.u_a + lane;
+    const uint32_t row = (uint32_t)(sink_end(g) + u * P.run_len - p0);
+    check_ok(u >= 0 && u < g.S && P.run_t0 + P.run_len <= g.T && row + (uint32_t)P.run_len <= (uint32_t)ROWS,
+             P.checks);
+    for (int ch = 0; ch < CHUNKS; ++ch)
+      tma_load_4d(dst + ch * (ROWS * 128) + row * 128u, box_map, bar, ch * 64, u, P.run_t0, head);
+  }
+  if ((f.gmask >> lane) & 1u) {
+    const int hrow = head * P.N;  // first row of the head in the [heads * N, d] view (fits: checked on the host)
+    int rr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      rr[i] = hrow + orig_index(g, min(p0 + 4 * lane + i, P.N - 1));
+      if (!check_ok(rr[i] >= hrow && rr[i] < hrow + P.N, P.checks)) rr[i] = hrow;
+    }
+    for (int ch = 0; ch < CHUNKS; ++ch)
+      tma_gather4(dst + ch * (ROWS * 128) + (uint32_t)lane * 512u, row_map, bar, ch * 64, rr[0], rr[1], rr[2], rr[3]);
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -250,8 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const uint32_t abort_addr = c.base + K::kAbortOff;
   int* status = P.status;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t t_start = P.cta_trace ? globaltimer_ns() : 0ull;
 
   if (threadIdx.x == 0) {
+    *reinterpret_cast<uint64_t*>(ctl_gen + K::kTraceOff) = 0ull;
     for (int st = 0; st < NS; ++st) {
       mbar_init(reinterpret_cast<uint64_t*>(ctl_gen) + st, 1);       // kv_full
       mbar_init(reinterpret_cast<uint64_t*>(ctl_gen) + NS + st, 1);  // kv_empty
@@ -307,42 +481,67 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // ------------------------------------------------------------------ producer
     // Lane 0 takes the waits, the work counter and the transaction counts; the results are
     // broadcast so that the whole warp follows the same control flow. Tiled loads are issued by
-    // lane 0; in fused token order a temporal item's rows are gathered, lane L fetching rows
-    // 4L .. 4L + 3 of each tile (their original indices) for both 64-column chunks.
-    uint32_t kv_pos = 0, q_iter = 0;
+    // lane 0; in fused token order a temporal item's tiles are read where their rows lie
+    // (fused_plan / fused_issue: whole runs as boxes by lanes 0.., edge groups gathered by lane L
+    // for rows 4L .. 4L + 3).
+    uint32_t kv_pos = 0, q_iter = 0, tr_items = 0, tr_tiles = 0;
     bool q_issued = false;
     for (uint32_t it = 0;; ++it) {
       const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
       if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.item_empty(slot), ph ^ 1u, abort_addr, status) : 0,
                        0))
         break;
-      const uint32_t idx = __shfl_sync(0xffffffffu, lane == 0 ? atomicAdd(P.counter, 1u) : 0u, 0);
-      const ItemInfo inf = decode_item<BK>(P, idx);
+      ItemInfo inf;
+      if (P.order == kOrderWork) {
+        int wc = 0;
+        uint32_t wpos = 0;
+        const bool got = lane == 0 ? claim_work_item(P, wc, wpos) : false;
+        const uint32_t code = __shfl_sync(0xffffffffu, got ? ((uint32_t)wc << 31) | wpos : 0xFFFFFFFFu, 0);
+        if (code == 0xFFFFFFFFu) {
+          memset(&inf, 0, sizeof(inf));
+        } else {
+          inf = decode_work_item(P, (int)(code >> 31), code & 0x7FFFFFFFu);
+        }
+      } else {
+        const uint32_t idx = __shfl_sync(0xffffffffu, lane == 0 ? atomicAdd(P.counter, 1u) : 0u, 0);
+        inf = decode_item<BK>(P, idx);
+      }
       if (lane == 0) {
         items[slot] = inf;
         mbar_arrive(c.item_full(slot));
+        if (inf.valid) {
+          ++tr_items;
+          tr_tiles += (uint32_t)(inf.nA + inf.nB);
+        }
       }
       if (!inf.valid) break;
       const bool gat = P.fused && inf.cls == SVG_ROUTE_TEMPORAL;
-      const MaskGeom& gg = P.g[SVG_ROUTE_TEMPORAL];
-      const int hrow = inf.head * P.N;  // first row of the head in the 2-D maps
       if (inf.nA + inf.nB > 0) {
         if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.q_free(), (q_iter & 1u) ^ 1u, abort_addr, status) : 0,
                          0))
           break;
         ++q_iter;
-        if (lane == 0) mbar_expect_tx(c.q_full(), (uint32_t)C::kQHalfBytes * ((inf.nA > 0) + (inf.nB > 0)));
+        FusedPlan qpl[2];
+        uint32_t qbytes = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if ((h == 0 ? inf.nA : inf.nB) == 0) continue;
+          if (gat) {
+            qpl[h] = fused_plan<kHalfRows>(P, inf.pair * kPairRows + h * kHalfRows, lane);
+            qbytes += fused_bytes<kHalfRows, C::kChunks>(P, qpl[h]);
+          } else {
+            qbytes += (uint32_t)C::kQHalfBytes;
+          }
+        }
+        if (lane == 0) mbar_expect_tx(c.q_full(), qbytes);
         __syncwarp();
+#pragma unroll
         for (int h = 0; h < 2; ++h) {
           if ((h == 0 ? inf.nA : inf.nB) == 0) continue;
           const int p0 = inf.pair * kPairRows + h * kHalfRows;
           if (gat) {
-            int rr[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) rr[i] = hrow + orig_index(gg, min(p0 + 4 * lane + i, P.N - 1));
-            for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_gather4(sQ + h * C::kQHalfBytes + ch * (128 * 128) + lane * 512, &P.tm_q2, c.q_full(), ch * 64, rr[0],
-                          rr[1], rr[2], rr[3]);
+            fused_issue<kHalfRows, C::kChunks>(P, qpl[h], &P.tm_q, &P.tm_q4, &P.tm_q2, sQ + h * C::kQHalfBytes,
+                                               c.q_full(), inf.head, p0, lane);
           } else if (lane == 0) {
             for (int ch = 0; ch < C::kQKChunks; ++ch)
               tma_load_3d(sQ + h * C::kQHalfBytes + ch * (128 * 128), &P.tm_q, c.q_full(), ch * C::kQKColsPerChunk, p0,
@@ -353,16 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       // K / V loads in the order the MMA warp consumes them: K(e), V(e) per entry; with P in
       // shared memory S(e+1) comes before P V(e): K(0), then K(e+1), V(e) per entry.
-      // the last two entries' key-tile row and gathered row indices, {entry, row0, rr[4]} by entry
-      // parity: each entry's are worked out once (static indices only, so they stay in registers)
-      int ca[6] = {-1, 0, 0, 0, 0, 0}, cb[6] = {-1, 0, 0, 0, 0, 0};
-      auto fill = [&](int (&cc)[6], int e) {
+      // the last two entries' key-tile rows, {entry, row0} by entry parity: each entry's is
+      // worked out once
+      int ca[2] = {-1, 0}, cb[2] = {-1, 0};
+      auto fill = [&](int (&cc)[2], int e) {
         cc[0] = e;
         cc[1] = (int)ent_kt(get_entry<BK>(P, inf, e)) * BK;
-        if (gat && 4 * lane < BK) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) cc[2 + i] = hrow + orig_index(gg, min(cc[1] + 4 * lane + i, P.N - 1));
-        }
       };
       bool ok = true;
       for (int n = 0; n < 2 * inf.count && ok; ++n) {
@@ -381,17 +576,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           e = (m >> 1) + ((m & 1) ^ 1);
           w = m & 1;
         }
-        int row0, rr[4];
+        int row0;
         if ((e & 1) == 0) {
           if (ca[0] != e) fill(ca, e);
           row0 = ca[1];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) rr[i] = ca[2 + i];
         } else {
           if (cb[0] != e) fill(cb, e);
           row0 = cb[1];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) rr[i] = cb[2 + i];
         }
         const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
         if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status) : 0,
@@ -399,14 +590,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           ok = false;
           break;
         }
-        if (lane == 0) mbar_expect_tx(c.kv_full(st), w == 0 ? C::kKBytes : C::kVBytes);
+        FusedPlan kpl;
+        if (gat) kpl = fused_plan<BK>(P, row0, lane);
+        if (lane == 0)
+          mbar_expect_tx(c.kv_full(st), gat ? fused_bytes<BK, C::kChunks>(P, kpl) : (w == 0 ? C::kKBytes : C::kVBytes));
         __syncwarp();
         const uint32_t dst = sRing + st * C::kTileBytes;
         if (gat) {
-          if (4 * lane < BK)
-            for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_gather4(dst + ch * (BK * 128) + lane * 512, w == 0 ? &P.tm_k2 : &P.tm_v2, c.kv_full(st), ch * 64,
-                          rr[0], rr[1], rr[2], rr[3]);
+          fused_issue<BK, C::kChunks>(P, kpl, w == 0 ? &P.tm_k : &P.tm_v, w == 0 ? &P.tm_k4 : &P.tm_v4,
+                                      w == 0 ? &P.tm_k2 : &P.tm_v2, dst, c.kv_full(st), inf.head, row0, lane);
         } else if (lane == 0) {
           if (w == 0) {
             for (int ch = 0; ch < C::kQKChunks; ++ch)
@@ -427,6 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         drain_bar(c.kv_full(pos % NS), (pos / NS) & 1u);
       }
       if (q_issued) drain_bar(c.q_full(), (q_iter - 1) & 1u);
+    }
+    if (lane == 0) {  // this CTA's share of the work, for the optional trace
+      *reinterpret_cast<uint32_t*>(ctl_gen + K::kTraceOff) = tr_items;
+      *reinterpret_cast<uint32_t*>(ctl_gen + K::kTraceOff + 4) = tr_tiles;
     }
   } else if (!skip_all && warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
@@ -653,8 +849,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       const int prow = in_range ? row : P.N - 1;
       // where the row lives in Q / O / LSE: its position, or its original index in fused order
       const int orow_idx = (P.fused && inf.cls == SVG_ROUTE_TEMPORAL) ? orig_index(P.g[SVG_ROUTE_TEMPORAL], prow) : prow;
+      const bool store_ok = check_ok(orow_idx >= 0 && orow_idx < P.N && inf.head >= 0 && inf.head < P.H, P.checks);
       if (nmine == 0) {  // no kept key for any row of this half (rounded masks only)
-        if (in_range) {
+        if (in_range && store_ok) {
           __nv_bfloat16* orow = P.o + ((size_t)inf.head * P.N + orow_idx) * D;
           const uint4 z = make_uint4(0, 0, 0, 0);
           for (int x = 0; x < D / 8; ++x) reinterpret_cast<uint4*>(orow)[x] = z;
@@ -743,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         tmem_ld32(tO + q * 32, o);
         tmem_ld_wait();
         tmem_ld_fence32(o);
-        if (in_range) {
+        if (in_range && store_ok) {
           uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
@@ -758,7 +955,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       tc_fence_before();
       mbar_arrive(c.o_free(h));
-      if (in_range && P.lse)
+      if (in_range && store_ok && P.lse)
         P.lse[(size_t)inf.head * P.N + orow_idx] =
             (l > 0.f && m != -INFINITY) ? (m * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
@@ -768,6 +965,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (P.cta_trace && threadIdx.x == 0 && (int)blockIdx.x < P.trace_ctas) {
+    unsigned long long* tr = P.cta_trace + 4 * (size_t)blockIdx.x;
+    tr[0] = t_start;
+    tr[1] = globaltimer_ns();
+    tr[2] = *reinterpret_cast<const uint32_t*>(ctl_gen + K::kTraceOff);
+    tr[3] = *reinterpret_cast<const uint32_t*>(ctl_gen + K::kTraceOff + 4);
+  }
 }
 
 // ---------------------------------------------------------------------------------------

@@ -24,8 +24,15 @@ constexpr uint32_t kTmMagic = 0x53564731u;  // "SVG1"
 constexpr int kMaxHeads = 4096;
 constexpr int64_t kMaxTokens = 1 << 22;
 constexpr int kPairRows = 256;  // query rows per item of the one-SM kernel: two 128-row halves
-constexpr int kQuadRows = 512;  // query rows per item of the two-SM kernel: 2 SMs x two halves
 constexpr int kHalfRows = 128;
+
+// Checked build (-DSVG_CHECKED=1, the library libsvgattn_checked.so): device-side bounds checks on
+// the indexes the kernels compute for global memory, tile-map arrays and TMA coordinates. A failed
+// check adds one to a device counter (svg_checks_failed reads it) and the access is skipped or its
+// index clamped into range; nothing traps. In the release build every check compiles away.
+#ifndef SVG_CHECKED
+#define SVG_CHECKED 0
+#endif
 
 // ---------------------------------------------------------------------------------------
 // Mask geometry in position space.
@@ -148,16 +155,16 @@ __host__ __device__ inline int row_kept_in(const MaskGeom& g, int lo, int hi, in
 // Tile-map workspace record (offset 0 of the workspace, 256 bytes).
 struct TmHeader {
   uint32_t magic, version;
-  int32_t T, H, W, route, k, b, F0, variant, layout, bq, bk, nq, nk, npairs, N, nquads;
+  int32_t T, H, W, route, k, b, F0, variant, layout, bq, bk, nq, nk, npairs, N;
   unsigned long long retained_exact, retained_map, n_full, n_boundary, n_empty, visited_area,
-      pair_entries, pair_half_tiles, quad_entries, quad_phase_tiles;
+      pair_entries, pair_half_tiles;
 };
 static_assert(sizeof(TmHeader) <= 256, "header must fit in 256 bytes");
 
 struct TmLayout {
   uint64_t total, cls, cnt, row_ptr, cols, pair_ptr, pair_ent, pair_cnt, pair_order;
-  uint64_t quad_ptr, quad_ent, quad_cnt, quad_order;
-  int nq, nk, npairs, nquads;
+  uint64_t pair_grp;
+  int nq, nk, npairs;
 };
 
 // Records a failed CUDA call (what + error) for svg_last_cuda_error; returns SVG_ERR_CUDA.
@@ -180,28 +187,24 @@ inline TmLayout tm_layout(int64_t N, int bq, int bk) {
   L.pair_ent = off;   off = align_up(off + 4 * (uint64_t)L.npairs * L.nk, 256);
   L.pair_cnt = off;   off = align_up(off + 8 * (uint64_t)L.npairs, 256);
   L.pair_order = off; off = align_up(off + 4 * (uint64_t)L.npairs, 256);
-  L.nquads = (int)((N + kQuadRows - 1) / kQuadRows);
-  L.quad_ptr = off;   off = align_up(off + 4 * (uint64_t)(L.nquads + 1), 256);
-  L.quad_ent = off;   off = align_up(off + 4 * (uint64_t)L.nquads * L.nk, 256);
-  L.quad_cnt = off;   off = align_up(off + 8 * (uint64_t)L.nquads, 256);
-  L.quad_order = off; off = align_up(off + 4 * (uint64_t)L.nquads, 256);
+  L.pair_grp = off;   off = align_up(off + 8 * (uint64_t)L.npairs, 256);
   L.total = off;
   return L;
 }
 
-// Execution-list entry of a group of G 128-row blocks (G = 2: pair, G = 4: quad):
-// kt in the low (32 - 2G) bits, then one 2-bit flag per block, block i at bit 32 - 2G + 2i.
-// In a quad, block i = 2 * rank + half (rank = SM of the pair, half = MMA phase).
+// Execution-list entry of a pair of 128-row blocks (a 256-row item): kt in the low 28 bits, then
+// one 2-bit flag per block, block i at bit 28 + 2i.
 enum : uint32_t { kFlagSkip = 0, kFlagFull = 1, kFlagMasked = 2, kFlagBounds = 3 };
 __host__ __device__ inline uint32_t ent_kt(uint32_t e) { return e & 0x0FFFFFFFu; }
 __host__ __device__ inline uint32_t ent_flag(uint32_t e, int half) { return (e >> (28 + 2 * half)) & 3u; }
-__host__ __device__ inline uint32_t qent_kt(uint32_t e) { return e & 0x00FFFFFFu; }
-__host__ __device__ inline uint32_t qent_flag(uint32_t e, int rank, int half) {
-  return (e >> (24 + 4 * rank + 2 * half)) & 3u;
-}
 
-// Scratch of the attention entry points: [0] status, [1] reserved, [2] work counter.
+// Scratch of the attention entry points: [0] status, [1] reserved, [2] work counter (head-major
+// order), bytes [16, 24): the two class positions of the work-ordered scheduler (low / high word).
 constexpr size_t kScratchBytes = 256;
+constexpr size_t kCounter64Off = 16;
+
+// Scheduling orders of the persistent attention kernel's work items.
+enum : int { kOrderHeadMajor = 0, kOrderWork = 1 };
 
 // Launch parameters of the attention kernel (filled on the host, read on the device).
 struct AttnParams {
@@ -210,6 +213,11 @@ struct AttnParams {
   // their rows with 4-row gathers through these 2-D maps ([heads * N] rows x d, box 64 x 1)
   // and write O rows back to their original index.
   CUtensorMap tm_q2, tm_k2, tm_v2;
+  // ... and through these 4-D maps (d, patch, frame, head) with a box of one patch x run_len frames:
+  // a whole run of one patch's frames (consecutive positions of a temporal head's order, rows S
+  // apart in the original order) in one tiled copy; run_len = 0 when runs are not copied as boxes
+  CUtensorMap tm_q4, tm_k4, tm_v4;
+  int run_len, run_t0;
   int fused;
   // QK^T operands in e4m3 (one byte per element): tm_q / tm_k then describe 1-byte tensors
   int qk8;
@@ -229,21 +237,36 @@ struct AttnParams {
   const uint32_t* pair_ent[2];
   const uint32_t* pair_cnt[2];
   const uint32_t* pair_order[2];
-  const uint32_t* quad_ptr[2];
-  const uint32_t* quad_ent[2];
-  const uint32_t* quad_cnt[2];
-  const uint32_t* quad_order[2];
-  int nquads;
+  // work-ordered scheduler: per position of pair_order, the [start, end) of its run of equal work
+  const uint32_t* pair_grp[2];
+  int order;  // kOrderHeadMajor or kOrderWork
+  int hc[2];  // heads of each route class
+  unsigned long long* counter64;
+  // nullable per-CTA trace, [trace_ctas][4]: start ns, end ns, items, 128-row half-tiles
+  unsigned long long* cta_trace;
+  int trace_ctas;
   int uses[2];
   int exp_T, exp_H, exp_W, exp_k, exp_b, exp_F0, exp_variant, exp_layout, exp_bq, exp_bk;
   int* status;
   unsigned int* counter;
+  unsigned int* checks;  // failed-check counter of the checked build (null in the release build)
   uint32_t route_bits[kMaxHeads / 32];
 };
 
 // ---------------------------------------------------------------------------------------
 // PTX wrappers.
 #if defined(__CUDACC__)
+// True when `ok` (always true in the release build); a false check is counted in *failed.
+__device__ __forceinline__ bool check_ok(bool ok, unsigned int* failed) {
+#if SVG_CHECKED
+  if (!ok && failed) atomicAdd(failed, 1u);
+  return ok;
+#else
+  (void)failed;
+  return true;
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -301,6 +324,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// 4-D tiled TMA load global -> shared of this CTA, completion counted on `bar` (bytes).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
+      "%6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 // Four rows r0..r3 (any order, any rows) of 64 columns starting at column c0 of a 2-D tensor
@@ -416,7 +448,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, M = 128 (one SM) or 256 (SM pair).
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, M = 128.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int n, bool b_mn_major, int m = 128) {
   return (1u << 4)                      // D format fp32
          | (1u << 7)                    // A format bf16
@@ -433,84 +465,6 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n, int m = 128) {
          | ((uint32_t)(m >> 4) << 24);  // M / 16
 }
 
-// ---- CTA pairs (clusters of 2) and the two-SM tensor-core forms ----
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// Shared::cluster address of the variable at shared address `a` in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Arrive (release, cluster scope) on an mbarrier given by its shared::cluster address.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t a) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t a, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-// TMA load into this CTA's shared memory whose completion is counted on an mbarrier of either
-// CTA of the pair (bar = shared::cluster address); the data lands in the issuing CTA only.
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
-                                                 int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-      "%5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// D (+)= A B over both SMs of the pair: each SM supplies 128 rows of A and half of B's N columns
-// (same shared-memory offsets in both), and receives its 128 rows of D in its own TMEM.
-__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// The mbarrier (shared::cluster address, in either CTA) arrives once all pair MMAs issued so
-// far by this thread have completed.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
 // ---- softmax arithmetic shared by the attention kernels ----
 __device__ __forceinline__ float ex2f(float x) {
   float y;
@@ -606,7 +560,8 @@ __device__ __forceinline__ void mask_scores(const AttnParams& P, int cls, uint32
       if (j >= nn) s[j] = -INFINITY;
   } else if (P.variant == SVG_MASK_ROUNDED) {
     const uint8_t* rcls = P.cls[cls] + (size_t)(prow / P.bq) * P.nk;
-    const bool rowkept = __ldg(rcls + ent_kt(ent)) == 1;
+    const bool in_map = check_ok(prow >= 0 && prow < P.N && ent_kt(ent) < (uint32_t)P.nk, P.checks);
+    const bool rowkept = in_map && __ldg(rcls + ent_kt(ent)) == 1;
 #pragma unroll
     for (int j = 0; j < BK; ++j)
       if (!(rowkept && j < nn)) s[j] = -INFINITY;

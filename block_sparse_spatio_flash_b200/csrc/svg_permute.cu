@@ -12,12 +12,15 @@
 
 namespace svg {
 
+unsigned int* checks_counter();
+
 struct PermParams {
   const uint4* in;
   uint4* out;
   int heads, N, row_vec;  // row_vec = 16-byte vectors per row (d*2/16)
   int inverse;
   MaskGeom g;             // route field ignored; per-head route from the bit set
+  unsigned int* checks;   // failed-check counter of the checked build
   uint32_t route_bits[kMaxHeads / 32];
 };
 
@@ -52,6 +55,7 @@ __global__ void __launch_bounds__(512) permute_kernel(const __grid_constant__ Pe
             src = ts_to_pos(g, t, r - t * g.S);
           }
         }
+        if (!check_ok(src >= 0 && src < P.N, P.checks)) src = 0;
         v[u] = __ldg(in + (int64_t)src * P.row_vec);
       }
     }
@@ -74,6 +78,7 @@ int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const
   P.row_vec = d * 2 / 16;
   P.inverse = inverse;
   P.g = make_geom(geom, mask, SVG_ROUTE_TEMPORAL);
+  P.checks = checks_counter();
   for (int h = 0; h < heads; ++h)
     if (h_route[h] == SVG_ROUTE_TEMPORAL) P.route_bits[h >> 5] |= 1u << (h & 31);
   // about 8 resident blocks per SM across all heads; each block moves >= 4 steps of rows

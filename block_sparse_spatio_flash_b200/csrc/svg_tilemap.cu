@@ -9,12 +9,15 @@
 //   * a CSR list of visited k-tiles per q-tile (the data structure the traversal walks);
 //   * per 256-row item (two 128-row halves, the attention kernel's unit of work) an entry
 //     list with one flag per half: skip / full / masked / full-but-ragged;
-//   * the items in descending order of work for the persistent scheduler.
+//   * the items in descending order of work for the persistent scheduler, with the bounds of each
+//     run of equal work.
 #include "svg_common.cuh"
 
 namespace svg {
 
-// Execution lists of groups of G 128-row blocks (pairs: G = 2, quads: G = 4).
+unsigned int* checks_counter();
+
+// Execution lists of groups of G 128-row blocks (pairs: G = 2, the attention kernel's items).
 struct GroupLists {
   uint32_t* ptr;    // [ngroups + 1]
   uint32_t* ent;    // [ngroups * nk]
@@ -32,8 +35,9 @@ struct TmParams {
   uint32_t* cnt;
   uint32_t* row_ptr;
   uint32_t* cols;
-  GroupLists pairs, quads;
+  GroupLists pairs;
   TmHeader* hdr;
+  unsigned int* checks;  // failed-check counter of the checked build
 };
 
 __device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v, unsigned long long* red) {
@@ -69,7 +73,7 @@ __global__ void __launch_bounds__(256) tm_classify(TmParams P, svg_geom geom, sv
     h->T = geom.frames; h->H = geom.grid_h; h->W = geom.grid_w; h->route = route;
     h->k = mask.frame_window; h->b = mask.spatial_band; h->F0 = mask.sink_frames;
     h->variant = mask.variant; h->layout = mask.layout; h->bq = tile.bq; h->bk = tile.bk;
-    h->nq = P.nq; h->nk = P.nk; h->npairs = P.npairs; h->N = g.N; h->nquads = P.quads.ngroups;
+    h->nq = P.nq; h->nk = P.nk; h->npairs = P.npairs; h->N = g.N;
   }
   __syncthreads();
   unsigned long long kept_tot = 0, map_tot = 0, nfull = 0, nbnd = 0, nemp = 0, varea = 0;
@@ -210,13 +214,11 @@ __global__ void __launch_bounds__(1024) tm_scan(TmParams P) {
   block_exclusive_scan(P.row_ptr, P.nq);
   __syncthreads();
   block_exclusive_scan(P.pairs.ptr, P.pairs.ngroups);
-  __syncthreads();
-  block_exclusive_scan(P.quads.ptr, P.quads.ngroups);
 }
 
-// Ordered compaction of one row of flags, 256 threads, chunk by chunk.
+// Ordered compaction of one row of flags, 256 threads, chunk by chunk, into out[0, cap).
 template <typename F>
-__device__ void compact_row(int n, uint32_t* out, F&& value_of) {
+__device__ void compact_row(int n, uint32_t* out, uint64_t cap, unsigned int* checks, F&& value_of) {
   __shared__ uint32_t wsum[8];
   __shared__ uint32_t base;
   if (threadIdx.x == 0) base = 0;
@@ -231,7 +233,10 @@ __device__ void compact_row(int n, uint32_t* out, F&& value_of) {
     __syncthreads();
     uint32_t off = base;
     for (int j = 0; j < w; ++j) off += wsum[j];
-    if (keep) out[off + __popc(bal & ((1u << l) - 1))] = v;
+    if (keep) {
+      const uint32_t at = off + __popc(bal & ((1u << l) - 1));
+      if (check_ok(at < cap, checks)) out[at] = v;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
       uint32_t tot = 0;
@@ -244,7 +249,9 @@ __device__ void compact_row(int n, uint32_t* out, F&& value_of) {
 __global__ void __launch_bounds__(256) tm_fill_cols(TmParams P) {
   const int qt = blockIdx.x;
   const uint8_t* row = P.cls + (size_t)qt * P.nk;
-  compact_row(P.nk, P.cols + P.row_ptr[qt], [&](int kt) -> uint32_t {
+  const uint32_t b0 = P.row_ptr[qt];
+  const uint64_t tiles = (uint64_t)P.nq * P.nk;
+  compact_row(P.nk, P.cols + b0, check_ok(b0 <= tiles, P.checks) ? tiles - b0 : 0, P.checks, [&](int kt) -> uint32_t {
     const uint8_t c = row[kt];
     return c ? ((uint32_t)kt | ((uint32_t)c << 30)) : 0xFFFFFFFFu;
   });
@@ -253,7 +260,9 @@ __global__ void __launch_bounds__(256) tm_fill_cols(TmParams P) {
 template <int G>
 __global__ void __launch_bounds__(256) tm_fill_groups(TmParams P, GroupLists L) {
   const int g = blockIdx.x;
-  compact_row(P.nk, L.ent + L.ptr[g], [&](int kt) -> uint32_t {
+  const uint32_t b0 = L.ptr[g];
+  const uint64_t cap = (uint64_t)L.ngroups * P.nk;
+  compact_row(P.nk, L.ent + b0, check_ok(b0 <= cap, P.checks) ? cap - b0 : 0, P.checks, [&](int kt) -> uint32_t {
     uint32_t ph;
     return group_entry<G>(P, g, kt, &ph);
   });
@@ -269,7 +278,34 @@ __global__ void tm_sort_groups(GroupLists L) {
     const uint32_t wq = L.cnt[2 * q] + L.cnt[2 * q + 1];
     rank += (wq > wp) || (wq == wp && q < p);
   }
-  L.order[rank] = (uint32_t)p;
+  if (rank < (uint32_t)L.ngroups) L.order[rank] = (uint32_t)p;
+}
+
+// For each position p of the pair order (descending work, ties by index), the bounds [start, end) of
+// the run of positions with the same work as p. The work-ordered scheduler of the attention kernel
+// hands out one run at a time for every head of a route class, head by head, so that the items in
+// flight at a time share each head's K / V rows.
+__global__ void tm_work_runs(GroupLists L, uint32_t* grp) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= L.ngroups) return;
+  auto work = [&](int i) -> uint32_t {
+    const uint32_t g = L.order[i];
+    return L.cnt[2 * g] + L.cnt[2 * g + 1];
+  };
+  const uint32_t w = work(p);
+  int lo = 0, hi = p;  // first position of the run: work is non-increasing along the order
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (work(mid) > w) lo = mid + 1; else hi = mid;
+  }
+  grp[2 * p] = (uint32_t)lo;
+  lo = p + 1;
+  hi = L.ngroups;  // first position after the run
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (work(mid) < w) hi = mid; else lo = mid + 1;
+  }
+  grp[2 * p + 1] = (uint32_t)lo;
 }
 
 int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* ws, cudaStream_t st) {
@@ -286,25 +322,22 @@ int build_tilemap(svg_geom geom, svg_mask mask, svg_tile tile, int route, void* 
   P.npairs = L.npairs;
   P.variant = mask.variant;
   P.hdr = reinterpret_cast<TmHeader*>(base);
+  P.checks = checks_counter();
   P.cls = base + L.cls;
   P.cnt = u32(L.cnt);
   P.row_ptr = u32(L.row_ptr);
   P.cols = u32(L.cols);
   P.pairs = GroupLists{u32(L.pair_ptr), u32(L.pair_ent), u32(L.pair_cnt), u32(L.pair_order), L.npairs,
                        &P.hdr->pair_entries, &P.hdr->pair_half_tiles};
-  P.quads = GroupLists{u32(L.quad_ptr), u32(L.quad_ent), u32(L.quad_cnt), u32(L.quad_order), L.nquads,
-                       &P.hdr->quad_entries, &P.hdr->quad_phase_tiles};
   cudaError_t e = cudaMemsetAsync(base, 0, 256, st);
   if (e != cudaSuccess) return record_cuda_error("cudaMemsetAsync(tile-map header)", e);
   tm_classify<<<L.nq, 256, 0, st>>>(P, geom, mask, tile, route);
   tm_group_count<2><<<L.npairs, 256, 0, st>>>(P, P.pairs);
-  tm_group_count<4><<<L.nquads, 256, 0, st>>>(P, P.quads);
   tm_scan<<<1, 1024, 0, st>>>(P);
   tm_fill_cols<<<L.nq, 256, 0, st>>>(P);
   tm_fill_groups<2><<<L.npairs, 256, 0, st>>>(P, P.pairs);
-  tm_fill_groups<4><<<L.nquads, 256, 0, st>>>(P, P.quads);
   tm_sort_groups<<<(L.npairs + 127) / 128, 128, 0, st>>>(P.pairs);
-  tm_sort_groups<<<(L.nquads + 127) / 128, 128, 0, st>>>(P.quads);
+  tm_work_runs<<<(L.npairs + 127) / 128, 128, 0, st>>>(P.pairs, u32(L.pair_grp));
   e = cudaGetLastError();
   return e == cudaSuccess ? SVG_OK : record_cuda_error("launch tile-map kernels", e);
 }

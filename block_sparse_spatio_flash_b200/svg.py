@@ -14,7 +14,9 @@ from typing import Optional, Sequence
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libsvgattn.so")
+# SVG_CHECKED=1 loads the checked build (device-side bounds checks, svg_checks_failed).
+_LIB_NAME = "libsvgattn_checked.so" if os.environ.get("SVG_CHECKED") == "1" else "libsvgattn.so"
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", _LIB_NAME)
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"{_LIB_PATH} is missing; build it with `python -m block_sparse_spatio_flash_b200.build`")
 _lib = ctypes.CDLL(_LIB_PATH)
@@ -48,21 +50,28 @@ class svg_tile(ctypes.Structure):
 
 class svg_tilemap_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in ("total_bytes", "cls", "cnt", "row_ptr", "cols", "pair_ptr",
-                                               "pair_ent", "pair_cnt", "pair_order", "quad_ptr", "quad_ent",
-                                               "quad_cnt", "quad_order")] + \
-               [(n, ctypes.c_int32) for n in ("nq", "nk", "npairs", "nquads")]
+                                               "pair_ent", "pair_cnt", "pair_order", "pair_grp")] + \
+               [(n, ctypes.c_int32) for n in ("nq", "nk", "npairs")]
+
+
+class svg_launch_opts(ctypes.Structure):
+    _fields_ = [("order", ctypes.c_int32), ("d_cta_trace", ctypes.c_void_p), ("trace_ctas", ctypes.c_int32)]
+
+
+SVG_ORDER_HEAD_MAJOR, SVG_ORDER_WORK = 0, 1
 
 
 class svg_tilemap_summary_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in ("retained_exact", "retained_map", "n_full", "n_boundary",
-                                               "n_empty", "visited_area", "pair_entries", "pair_half_tiles",
-                                               "quad_entries", "quad_phase_tiles")]
+                                               "n_empty", "visited_area", "pair_entries", "pair_half_tiles")]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 _u8p = ctypes.POINTER(ctypes.c_uint8)
 _sig = {
     "svg_version": (ctypes.c_int, []),
+    "svg_checked_build": (ctypes.c_int, []),
+    "svg_checks_failed": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _i32]),
     "svg_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "svg_last_cuda_error": (ctypes.c_char_p, []),
     "svg_tilemap_bytes": (_sz, [svg_geom, svg_tile]),
@@ -85,6 +94,9 @@ _sig = {
                                                _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
     "svg_attention_fwd_qk8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp,
                                              _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
+    "svg_attention_fwd_ex": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p, _vp,
+                                            _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp,
+                                            ctypes.POINTER(svg_launch_opts), _vp]),
     "svg_test_attention_fwd_stall": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, ctypes.c_float, _u8p,
                                                     _vp, _vp, svg_geom, svg_mask, svg_tile, _i32, _vp, _sz, _vp, _vp]),
     "svg_attention_host_buffer_bytes": (_sz, [_i64, _i32, _i32]),
@@ -145,6 +157,17 @@ def make_tile(bq, bk) -> svg_tile:
 # ------------------------------------------------------------------------------ entry points
 def svg_version() -> int:
     return _lib.svg_version()
+
+
+def svg_checked_build() -> bool:
+    return bool(_lib.svg_checked_build())
+
+
+def svg_checks_failed(reset: bool = True) -> int:
+    """Failed device-side bounds checks since the last reset (checked build; 0 otherwise)."""
+    n = ctypes.c_uint32(0)
+    _check(_lib.svg_checks_failed(ctypes.byref(n), 1 if reset else 0), "svg_checks_failed")
+    return int(n.value)
 
 
 def svg_error_string(code: int) -> str:
@@ -218,6 +241,23 @@ def svg_attention_fwd_qk8(q8, k8, v, o, routes, ws_spatial, ws_temporal, geom, m
                                       _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile, mode,
                                       _ptr(scratch), scratch.numel() * scratch.element_size(), _ptr(status),
                                       _stream(stream)), "svg_attention_fwd_qk8")
+    return o
+
+
+def svg_attention_fwd_ex(q, k, v, o, routes, ws_spatial, ws_temporal, geom, mask, tile, mode=SVG_MODE_SPLIT,
+                         scratch=None, lse=None, scale: float = 0.0, status=None, order=SVG_ORDER_HEAD_MAJOR,
+                         cta_trace=None, stream=None) -> torch.Tensor:
+    """svg_attention_fwd with a scheduling order and an optional per-CTA trace (device int64 tensor
+    [n, 4]: start ns, end ns, items, half-tiles per CTA)."""
+    heads, tokens, d = q.shape
+    opts = svg_launch_opts(order, None if cta_trace is None else cta_trace.data_ptr(),
+                           0 if cta_trace is None else cta_trace.shape[0])
+    if cta_trace is not None:
+        _ptr(cta_trace)
+    _check(_lib.svg_attention_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), heads, tokens, d, scale,
+                                     _routes(routes), _ptr(ws_spatial), _ptr(ws_temporal), geom, mask, tile, mode,
+                                     _ptr(scratch), scratch.numel() * scratch.element_size(), _ptr(status),
+                                     ctypes.byref(opts), _stream(stream)), "svg_attention_fwd_ex")
     return o
 
 
@@ -333,9 +373,6 @@ def tilemap_arrays(ws: torch.Tensor, geom: svg_geom, tile: svg_tile) -> dict:
         "pair_ent": u32(L.pair_ent, np_ * nk),
         "pair_cnt": u32(L.pair_cnt, 2 * np_).view(np_, 2),
         "pair_order": u32(L.pair_order, np_),
-        "quad_ptr": u32(L.quad_ptr, L.nquads + 1),
-        "quad_ent": u32(L.quad_ent, L.nquads * nk),
-        "quad_cnt": u32(L.quad_cnt, 2 * L.nquads).view(L.nquads, 2),
-        "quad_order": u32(L.quad_order, L.nquads),
-        "nq": nq, "nk": nk, "npairs": np_, "nquads": L.nquads,
+        "pair_grp": u32(L.pair_grp, 2 * np_).view(np_, 2),
+        "nq": nq, "nk": nk, "npairs": np_,
     }

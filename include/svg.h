@@ -39,10 +39,9 @@
  *     built for other parameters) are written to the status word (see svg_read_status).
  *   - Requires a compute capability 10.0 device (B200, sm_100a); otherwise
  *     SVG_ERR_UNSUPPORTED.
- *   - Environment (read once per process by the host code): SVG_KERNEL=pair or SVG_KERNEL=pair1
- *     makes d = 128 attention run on the two-SM kernels instead of the one-SM kernel, and
- *     SVG_KERNEL=ps makes the one-SM kernel stage P in shared memory instead of tensor memory,
- *     each with the same results up to rounding.
+ *   - Environment (read once per process by the host code): SVG_KERNEL=ps makes the attention
+ *     kernel stage P in shared memory instead of tensor memory (the same results up to
+ *     rounding), for every attention entry point.
  *   - Per-device state (the streams of svg_attention_fwd_host, device attributes) is created on
  *     first use and belongs to the device's primary context: do not reset a device
  *     (cudaDeviceReset) while the library is in use on it.
@@ -94,11 +93,9 @@ typedef struct {
     uint64_t pair_ent;    /* uint32 [...]     kt | flagA << 28 | flagB << 30                  */
     uint64_t pair_cnt;    /* uint32 [2*np]    active entries of half 0 / half 1 of each pair  */
     uint64_t pair_order;  /* uint32 [np]      pairs by descending work, ties by index         */
-    uint64_t quad_ptr;    /* uint32 [nquad+1] offsets of the 512-row (two-SM) execution lists  */
-    uint64_t quad_ent;    /* uint32 [...]     kt | flag(rank r, half h) << (24 + 4r + 2h)      */
-    uint64_t quad_cnt;    /* uint32 [2*nquad] entries where MMA phase 0 / phase 1 is active     */
-    uint64_t quad_order;  /* uint32 [nquad]   quads by descending work, ties by index           */
-    int32_t nq, nk, npairs, nquads;
+    uint64_t pair_grp;    /* uint32 [2*np]    per position of pair_order: [start, end) of its run
+                                              of positions with equal work                      */
+    int32_t nq, nk, npairs;
 } svg_tilemap_layout;
 
 /* Totals of one built tile map (svg_tilemap_summary). */
@@ -109,8 +106,6 @@ typedef struct {
     uint64_t visited_area;    /* in-range pairs inside non-empty tiles                     */
     uint64_t pair_entries;    /* entries of all 256-row execution lists                    */
     uint64_t pair_half_tiles; /* active (entry, half) combinations: MMA work units          */
-    uint64_t quad_entries;    /* entries of all 512-row execution lists                    */
-    uint64_t quad_phase_tiles;/* active (entry, phase) combinations of the 512-row lists    */
 } svg_tilemap_summary_t;
 
 /*
@@ -126,10 +121,10 @@ int svg_tilemap_get_layout(svg_geom geom, svg_tile tile, svg_tilemap_layout *out
  * Classifies every (query tile, key tile) pair of one route class as full / boundary /
  * empty (rounded variant: full / empty), counts retained pairs per tile exactly, and
  * builds: the per-q-tile CSR list of visited tiles; the execution lists used by
- * svg_attention_fwd, one per group of 128-row query blocks -- pairs (256 rows, one SM) and
- * quads (512 rows, two SMs) -- with a flag per block: 0 skip, 1 full, 2 masked, 3 full but
- * key range past the sequence end; and the group orders by descending work used by the
- * persistent scheduler. Integer work only.
+ * svg_attention_fwd, one per pair of 128-row query blocks (256 rows, the kernel's work item),
+ * with a flag per block: 0 skip, 1 full, 2 masked, 3 full but key range past the sequence end;
+ * and the pairs in descending order of work, with the runs of equal work, for the persistent
+ * scheduler. Integer work only.
  *   d_ws: device buffer of at least svg_tilemap_bytes(geom, tile) bytes, 256-B aligned;
  *         written entirely by this call (also records the parameters it was built for).
  * Errors: SVG_ERR_ARG (bad geometry/mask/route), SVG_ERR_UNSUPPORTED (tile shape),
@@ -181,6 +176,34 @@ int svg_attention_fwd(const void *q, const void *k, const void *v, void *o, floa
                       const uint8_t *h_route, const void *d_ws_spatial, const void *d_ws_temporal,
                       svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
                       void *d_scratch, size_t scratch_bytes, int32_t *d_status, void *stream);
+
+/*
+ * Scheduling and tracing options of svg_attention_fwd_ex.
+ *   order: SVG_ORDER_HEAD_MAJOR hands the persistent CTAs the work items (256 query rows of one head)
+ *          head by head, each head's items heaviest first -- the order of svg_attention_fwd.
+ *          SVG_ORDER_WORK hands them out by descending work over ALL heads (longest processing time
+ *          first): every head of a route class has the same items, so each class's items are taken
+ *          run by run of equal work, head by head within a run, and the two classes are merged by
+ *          work. Results are identical; only which CTA computes which rows, and when, changes.
+ *   d_cta_trace: nullable device uint64 [trace_ctas][4]; when given, the call clears it and each CTA
+ *          i < trace_ctas of the launch writes {start ns, end ns (%globaltimer), items it ran, 128-row
+ *          half-tiles of those items}. Give trace_ctas >= the device's SM count to see every CTA;
+ *          entries of CTAs that did not run stay 0. 8-byte aligned.
+ */
+enum { SVG_ORDER_HEAD_MAJOR = 0, SVG_ORDER_WORK = 1 };
+typedef struct {
+    int32_t order;
+    uint64_t *d_cta_trace;
+    int32_t trace_ctas;
+} svg_launch_opts;
+
+/* svg_attention_fwd with the options above (opts must not be NULL: SVG_ERR_ARG). */
+int svg_attention_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int32_t heads, int64_t tokens, int32_t d, float scale,
+                         const uint8_t *h_route, const void *d_ws_spatial, const void *d_ws_temporal,
+                         svg_geom geom, svg_mask mask, svg_tile tile, int32_t mode,
+                         void *d_scratch, size_t scratch_bytes, int32_t *d_status,
+                         const svg_launch_opts *opts, void *stream);
 
 /*
  * svg_attention_fwd with QK^T on the tensor core's 8-bit path: q8 and k8 are e4m3 (one byte per
@@ -329,6 +352,18 @@ const char *svg_error_string(int code);
 /* Which CUDA call last failed on the calling thread and why (after an SVG_ERR_CUDA return);
  * "none" if none has. The string stays valid until the next failing call on that thread. */
 const char *svg_last_cuda_error(void);
+
+/*
+ * Checked build (libsvgattn_checked.so, compiled with -DSVG_CHECKED=1): every kernel checks the
+ * indexes it computes for global memory, tile-map arrays and TMA coordinates; a failed check is
+ * counted in a device counter and the access is skipped or clamped into range (no trap). For debug
+ * runs on small cases; the release build compiles the checks away.
+ *   svg_checked_build(): 1 in the checked build, 0 in the release build.
+ *   svg_checks_failed(): failed checks since the last reset into *h_count, cleared when reset != 0;
+ *     synchronises the device. The release build sets *h_count = 0 without touching the device.
+ */
+int svg_checked_build(void);
+int svg_checks_failed(uint32_t *h_count, int32_t reset);
 
 /* Library version (major*10000 + minor*100 + patch). */
 int svg_version(void);

@@ -59,12 +59,10 @@ def test_tilemap_layout_sizes(svg):
         n = 21 * 45 * 80
         assert L.nq == -(-n // bq) and L.nk == -(-n // bk) and L.npairs == -(-n // 256)
         assert L.total_bytes == svg.svg_tilemap_bytes(g, t)
-        offs = [L.cls, L.cnt, L.row_ptr, L.cols, L.pair_ptr, L.pair_ent, L.pair_cnt, L.pair_order,
-                L.quad_ptr, L.quad_ent, L.quad_cnt, L.quad_order]
-        assert L.nquads == -(-n // 512)
+        offs = [L.cls, L.cnt, L.row_ptr, L.cols, L.pair_ptr, L.pair_ent, L.pair_cnt, L.pair_order, L.pair_grp]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert L.cnt - L.cls >= L.nq * L.nk and L.pair_ent - L.pair_ptr >= 4 * (L.npairs + 1)
-        assert L.total_bytes >= L.quad_order + 4 * L.nquads
+        assert L.pair_grp >= L.pair_order + 4 * L.npairs and L.total_bytes >= L.pair_grp + 8 * L.npairs
 
 
 def test_bad_tile_and_geometry_rejected(svg):

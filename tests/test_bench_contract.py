@@ -62,3 +62,18 @@ def test_clock_sampler_writes_outside_the_repository(tmp_path):
     assert not c.path.startswith(bench.ROOT)
     c2 = bench.ClockSampler(0, str(tmp_path))
     assert c2.path.startswith(str(tmp_path))
+
+
+def test_trace_stats_of_a_synthetic_trace():
+    import torch
+    # three CTAs: busy 4, 6 and 10 ms from a common start; a fourth entry never ran (zeros)
+    t0 = 1_000_000_000
+    tr = torch.tensor([[t0, t0 + 4_000_000, 3, 30], [t0, t0 + 6_000_000, 4, 40], [t0, t0 + 10_000_000, 5, 50],
+                       [0, 0, 0, 0]], dtype=torch.int64)
+    s = bench.trace_stats(tr)
+    assert s["ctas"] == 3 and abs(s["span_ms"] - 10.0) < 1e-9
+    assert abs(s["busy_max_ms"] - 10.0) < 1e-9 and abs(s["busy_mean_ms"] - 20.0 / 3) < 1e-9
+    assert abs(s["tail_ms"] - 4.0) < 1e-9  # last end 10 ms, median end 6 ms
+    assert abs(s["idle_frac"] - (1 - 20.0 / 30.0)) < 1e-9
+    assert (s["tiles_max"], s["tiles_min"], s["items_max"], s["items_min"]) == (50, 30, 5, 3)
+    assert bench.trace_stats(torch.zeros((2, 4), dtype=torch.int64)) is None

@@ -31,9 +31,10 @@ def u32(t):
 
 
 def expected_group_entries(cls, N, bq, bk, G):
-    """Execution lists derived from the class map for groups of G 128-row blocks (G = 2: pairs,
-    G = 4: quads). Block flag: 0 skip, 1 full, 2 masked, 3 full but ragged key tile; block i of a
-    group sits at bit 32 - 2G + 2i; per group, the entries in which MMA phase i % 2 is active."""
+    """Execution lists derived from the class map for groups of G 128-row blocks (G = 2: the pairs
+    of the kernel's 256-row items). Block flag: 0 skip, 1 full, 2 masked, 3 full but ragged key
+    tile; block i of a group sits at bit 32 - 2G + 2i; per group, the entries in which block i is
+    active."""
     nq, nk = cls.shape
     rows = 128 * G
     ngroups = -(-N // rows)
@@ -66,7 +67,7 @@ def expected_group_entries(cls, N, bq, bk, G):
 
 
 def check_group_lists(A, summ, cls, N, bq, bk, G):
-    key = "pair" if G == 2 else "quad"
+    key = "pair"
     ents, cnts = expected_group_entries(cls, N, bq, bk, G)
     ptr = u32(A[key + "_ptr"]).astype(np.int64)
     ent = u32(A[key + "_ent"])
@@ -77,8 +78,14 @@ def check_group_lists(A, summ, cls, N, bq, bk, G):
     work = cnt.sum(axis=1).astype(np.int64)
     order = u32(A[key + "_order"]).astype(np.int64)
     assert np.array_equal(order, np.lexsort((np.arange(len(work)), -work)))
-    tot_e = summ.pair_entries if G == 2 else summ.quad_entries
-    tot_w = summ.pair_half_tiles if G == 2 else summ.quad_phase_tiles
+    if G == 2:  # runs of equal work along the order, for the work-ordered scheduler
+        ws = work[order]
+        grp = u32(A["pair_grp"]).astype(np.int64).reshape(-1, 2)
+        for p_ in range(len(ws)):
+            same = np.nonzero(ws == ws[p_])[0]
+            assert grp[p_, 0] == same[0] and grp[p_, 1] == same[-1] + 1, (p_, grp[p_], same[[0, -1]])
+    tot_e = summ.pair_entries
+    tot_w = summ.pair_half_tiles
     assert tot_e == sum(len(e) for e in ents) and tot_w == int(work.sum())
 
 
@@ -123,7 +130,6 @@ def check_tilemap(S, w, route, variant, bq, bk, qts=None):
         assert np.array_equal(seg >> 30, cls[qt, kts])
     # execution lists and scheduler orders (derived from the map, which matched the oracle)
     check_group_lists(A, summ, cls, N, bq, bk, 2)
-    check_group_lists(A, summ, cls, N, bq, bk, 4)
     return summ
 
 
@@ -481,6 +487,51 @@ def test_fused_order_pages_mixed(S):
     got, _, st = gp.run_fused(w, q, k, v, lse=False)
     assert st == 0
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- scheduling order
+def _run_ordered(S, w, qp, kp, vp, maps, g, m, t, order, mode=0):
+    o = torch.empty_like(qp)
+    ls = torch.empty(qp.shape[:2], dtype=torch.float32, device=qp.device)
+    sc = S.alloc_scratch()
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    tr = torch.full((n + 3, 4), -1, dtype=torch.int64, device=qp.device)
+    S.svg_attention_fwd_ex(qp, kp, vp, o, list(w.routes), maps[0], maps[1], g, m, t, mode=mode, scratch=sc, lse=ls,
+                           order=order, cta_trace=tr)
+    assert S.svg_read_status(sc) == 0
+    return o, ls, tr.cpu()
+
+
+@pytest.mark.parametrize("w,variant", [(MEDIUM, 0), (MEDIUM.replace(routes=(1, 1, 0, 1, 0, 0, 1)), 1),
+                                       (syn.MIXED_75K, 0)], ids=["medium", "medium7_rounded", "mixed_75600"])
+def test_work_order_gives_the_same_bytes_and_a_complete_trace(S, w, variant):
+    """The work-ordered scheduler (longest processing time first over all heads) computes exactly the
+    head-major order's bytes; the per-CTA trace accounts for every item and half-tile once."""
+    g, m, t = gp.geom_mask_tile(w, variant)
+    routes = list(w.routes)
+    q, k, v = (x.cuda() for x in syn.make_qkv(w, seed_offset=71))
+    qp, kp, vp = (torch.empty_like(x) for x in (q, k, v))
+    for a, b in ((q, qp), (k, kp), (v, vp)):
+        S.svg_permute(a, b, routes, g, m)
+    maps = gp.build_maps(w, g, m, t, routes)
+    summ = {c: S.svg_tilemap_summary(maps[c]) for c in (0, 1) if maps[c] is not None}
+    o0, l0, tr0 = _run_ordered(S, w, qp, kp, vp, maps, g, m, t, S.SVG_ORDER_HEAD_MAJOR)
+    o1, l1, tr1 = _run_ordered(S, w, qp, kp, vp, maps, g, m, t, S.SVG_ORDER_WORK)
+    assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+    assert torch.equal(l0, l1)
+    npairs = -(-w.tokens // 256)
+    want_tiles = sum(summ[r].pair_half_tiles for r in routes)
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    for tr in (tr0, tr1):
+        ran = tr[:n][tr[:n, 2] > 0]
+        assert int(tr[:n, 2].sum()) == w.heads * npairs and int(tr[:n, 3].sum()) == want_tiles
+        assert (ran[:, 1] >= ran[:, 0]).all() and (ran[:, 0] > 0).all()
+        assert (tr[n:] == 0).all()  # entries past the grid are cleared and never written
+    if w.tokens > 10000:  # and against the oracle on sampled rows
+        out = torch.empty_like(o1)
+        S.svg_permute(o1, out, routes, g, m, inverse=True)
+        q0, k0, v0 = syn.make_qkv(w, seed_offset=71)
+        gp.compare_rows(w.replace(sample_rows=128), q0, k0, v0, out.cpu(), None)
 
 
 # ----------------------------------------------------------------------------- limits

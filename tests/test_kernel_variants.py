@@ -1,8 +1,8 @@
-"""The selectable kernels (SVG_KERNEL=pair: 512-row items, two halves per SM; SVG_KERNEL=pair1:
-one 128-row half per SM, key tiles alternating between two softmax groups; SVG_KERNEL=ps: the
-single-SM kernel with P staged in shared memory) against the oracle, on every entry the option
-reaches: sparse (both modes, both masks), dense, d = 64, fused token order, and for ps the e4m3 QK^T
-call and the bounded-wait path. The kernel choice is read once per process, so each runs in a child process."""
+"""The selectable schedule (SVG_KERNEL=ps: the attention kernel with P staged in shared memory)
+against the oracle, on every entry the option reaches: sparse (both modes, both masks), dense,
+d = 64, fused token order (bitwise equal to the permuted path under the same schedule), e4m3
+QK^T and the bounded-wait path. The choice is read once per process, so it runs in a child
+process."""
 import os
 import subprocess
 import sys
@@ -54,24 +54,22 @@ got, _, st2 = gp.run_fused(wf, q, k, v, lse=False)
 assert st == 0 and st2 == 0, (st, st2)
 assert (got.view(torch.int16) == want.view(torch.int16)).all()
 gp.compare_rows(wf, q, k, v, got, None)
-if {one_sm}:  # the two-SM options leave the e4m3 call and the stall hook to the one-SM kernel
-    q8, k8 = gp.quantize_e4m3(q), gp.quantize_e4m3(k)
-    out, st = gp.run_qk8(wf, q8, k8, v)
-    assert st == 0, st
-    gp.compare_rows(wf, q8, k8, v, out, None)
-    _, _, st = gp.run_path(wf, q, k, v, stall=True)
-    assert st == -4, st
-    out, lse, st = gp.run_path(wf, q, k, v)
-    assert st == 0, st
-    gp.compare_rows(wf, q, k, v, out, lse)
+q8, k8 = gp.quantize_e4m3(q), gp.quantize_e4m3(k)
+out, st = gp.run_qk8(wf, q8, k8, v)
+assert st == 0, st
+gp.compare_rows(wf, q8, k8, v, out, None)
+_, _, st = gp.run_path(wf, q, k, v, stall=True)
+assert st == -4, st
+out, lse, st = gp.run_path(wf, q, k, v)
+assert st == 0, st
+gp.compare_rows(wf, q, k, v, out, lse)
 print("ok")
 """
 
 
-@pytest.mark.parametrize("kernel", ["pair", "pair1", "ps"])
-def test_two_sm_kernels_match_oracle(kernel):
-    env = dict(os.environ, SVG_KERNEL=kernel)
-    child = CHILD.format(root=ROOT, one_sm=kernel == "ps")
+def test_p_in_shared_memory_schedule_matches_oracle():
+    env = dict(os.environ, SVG_KERNEL="ps")
+    child = CHILD.format(root=ROOT)
     r = subprocess.run([sys.executable, "-c", child], env=env, cwd=ROOT, capture_output=True,
                        text=True, timeout=600)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), (r.stdout[-2000:], r.stderr[-4000:])
