@@ -17,8 +17,8 @@ int launch_permute(const void* in, void* out, int heads, int64_t N, int d, const
                    svg_mask mask, int inverse, int num_sms, cudaStream_t st);
 int launch_attention(const AttnParams& P, int d, int bk, int grid, bool p_smem, cudaStream_t st);
 size_t route_work_bytes(int heads, int64_t N, int d, int n_rows);
-int launch_route(const void* q, const void* k, const void* v, int heads, int N, int d, float scale, svg_geom geom,
-                 svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
+int launch_route(const void* q, const CUtensorMap* tm_k, const CUtensorMap* tm_v, int heads, int N, int d, float scale,
+                 svg_geom geom, svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
                  int num_sms, cudaStream_t st);
 }  // namespace svg
 
@@ -29,8 +29,10 @@ int record_cuda_error(const char* what, int cuda_error);
 unsigned int* checks_counter();
 }
 
+#if SVG_CHECKED
 // Failed-check counter of the checked build (see SVG_CHECKED in svg_common.cuh).
 static __device__ unsigned int g_checks_failed;
+#endif
 
 // Device address of the counter (null in the release build, whose kernels never use it).
 unsigned int* svg::checks_counter() {
@@ -557,7 +559,7 @@ int svg_route_heads(const void* q, const void* k, const void* v, int32_t heads, 
                     svg_geom geom, svg_mask mask, const int32_t* d_rows, int32_t n_rows, void* d_work,
                     size_t work_bytes, uint8_t* d_route, float* d_err, void* stream) {
   if (!q || !k || !v || !d_rows || !d_work || !d_route) return SVG_ERR_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(d_rows, 4) || !aligned(d_work, 4) ||
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(d_rows, 4) || !aligned(d_work, 256) ||
       (d_err && !aligned(d_err, 4)))
     return SVG_ERR_ARG;
   if (heads < 1 || heads > 65535 || n_rows < 1 || !geom_ok(geom) || !mask_ok(geom, mask)) return SVG_ERR_ARG;
@@ -568,7 +570,10 @@ int svg_route_heads(const void* q, const void* k, const void* v, int32_t heads, 
   int rc = device_info(&num_sms);
   if (rc) return rc;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
-  return launch_route(q, k, v, heads, (int)tokens, d, sc, geom, mask, d_rows, n_rows, d_work, d_route, d_err,
+  CUtensorMap tmk, tmv;  // K / V tiles of 64 keys for the tensor-core kernel
+  if ((rc = encode_qkv_map(&tmk, k, heads, (int)tokens, d, 64))) return rc;
+  if ((rc = encode_qkv_map(&tmv, v, heads, (int)tokens, d, 64))) return rc;
+  return launch_route(q, &tmk, &tmv, heads, (int)tokens, d, sc, geom, mask, d_rows, n_rows, d_work, d_route, d_err,
                       num_sms, static_cast<cudaStream_t>(stream));
 }
 

@@ -32,7 +32,6 @@ namespace svg {
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 
 // QK8: Q and K in e4m3 (one byte per element, d = 128: one 128-byte swizzle chunk per row), QK^T on
@@ -109,45 +108,6 @@ struct Ctl {
   static constexpr uint32_t kBytes = kTraceOff + 8;
 };
 
-__device__ __forceinline__ int ld_shared_volatile(uint32_t addr) {
-  int v;
-  asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_shared(uint32_t addr, int v) {
-  asm volatile("st.volatile.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-// Bounded wait on an mbarrier phase. Returns false on timeout or when another role aborted.
-// abort_addr: shared address of the abort flag; status: global status word.
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr, int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0) {
-      if (ld_shared_volatile(abort_addr)) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        st_shared(abort_addr, 1);
-        atomicCAS(status, 0, SVG_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// Fast path inline (an already-completed phase costs one try_wait), the bounded loop out of line.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t abort_addr, int* status) {
-  return mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, abort_addr, status);
-}
-
-// Drain wait: ignores the abort flag, short limit; used only on the error path.
-__device__ __noinline__ void drain_bar(uint32_t a, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, parity))
-    if (globaltimer_ns() - t0 > 200000000ull) return;
-}
-
 // O_h *= alpha in TMEM, 32 columns at a time (one thread per row).
 template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
@@ -161,30 +121,6 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
     for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
     tmem_st32(tO + q * 32, o);
   }
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-// Makes this thread's shared-memory stores visible to the tensor core (the async proxy).
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// One P row (BK bf16, packed in pairs in r[0, BK/2)) into a K-major 128-byte-swizzle tile of
-// 128 rows: keys [64c, 64c + 64) in chunk c (128 rows x 128 bytes), row lr at byte lr * 128 of the
-// chunk, its 16-byte unit u at position u ^ (lr % 8). A warp's 32 rows cover all banks in four
-// passes per store.
-template <int BK>
-__device__ __forceinline__ void store_p_sw128(uint32_t base, int lr, const uint32_t* r) {
-  const uint32_t row = base + (uint32_t)lr * 128u, sw = (uint32_t)lr & 7u;
-#pragma unroll
-  for (int ch = 0; ch < BK / 64; ++ch)
-#pragma unroll
-    for (uint32_t u = 0; u < 8; ++u) {
-      const uint32_t* w = r + ch * 32 + 4 * u;
-      st_shared_v4(row + ch * (128u * 128u) + ((u ^ sw) << 4), w[0], w[1], w[2], w[3]);
-    }
 }
 
 template <int BK>

@@ -7,23 +7,20 @@
 // the sparse mask whose outputs are closer to the dense ones (relative squared error over the
 // sampled rows; ties go to spatial).
 //
-// route_partial_kernel: one block = 32 sampled rows of one head x one chunk of the keys. K/V tiles
-// of 64 keys are staged in shared memory as bf16; warp w owns rows 4w..4w+3 and keeps, per row and
-// mask (dense / spatial / temporal), an online softmax in fp32 on the CUDA cores: scores with keys
-// lane and lane + 32 (register-blocked 4 rows x 2 keys), then P V with output dims
-// [lane * D/32, (lane + 1) * D/32). The unnormalised state (O, running max, running sum) of each
-// chunk is written out; route_merge_kernel combines the chunks of a row and writes
+// route_tc_kernel (tensor cores, below): one CTA = up to 128 sampled rows of one head x one chunk of
+// the keys; per row and mask (dense / spatial / temporal) an online softmax, the scores and the three
+// P V products on tcgen05. The unnormalised state (O, running max, running sum) of each chunk is
+// written out; route_merge_kernel combines the chunks of a row and writes
 // (|O_s - O_d|^2, |O_t - O_d|^2, |O_d|^2); route_reduce_kernel sums those per head in a fixed
 // order (deterministic) and sets the route.
 #include <cuda_bf16.h>
+#include <string.h>
 
 #include "svg_common.cuh"
 
 namespace svg {
 
-constexpr int kRouteRows = 32;      // sampled rows per block (4 per warp)
-constexpr int kRouteKeys = 64;      // keys per shared-memory tile
-constexpr int kRouteThreads = 256;
+constexpr int kRouteKeys = 64;      // keys per tile
 constexpr int kRouteMaxChunks = 32;
 constexpr int kRouteChunkKeys = 2048;
 
@@ -38,11 +35,11 @@ inline int route_chunk_len(int64_t N, int G) {
   return (int)((per + kRouteKeys - 1) / kRouteKeys * kRouteKeys);
 }
 // Chunks for this launch: the count (at most route_chunks(N), the count the work buffer is sized
-// for) whose blocks fill the GPU's 2 x SM block slots best over whole waves -- a last, mostly empty
-// wave costs as much as a full one; among equals the larger count (shorter blocks).
-inline int route_launch_chunks(int64_t N, int row_blocks, int heads, int num_sms) {
+// for) whose blocks fill the GPU's block slots (blocks_per_sm x SMs) best over whole waves -- a
+// last, mostly empty wave costs as much as a full one; among equals the larger count (shorter blocks).
+inline int route_launch_chunks(int64_t N, int row_blocks, int heads, int num_sms, int blocks_per_sm) {
   const int64_t per_chunk = (int64_t)row_blocks * heads;
-  const int64_t slots = 2 * (int64_t)(num_sms > 0 ? num_sms : 1);
+  const int64_t slots = (int64_t)blocks_per_sm * (num_sms > 0 ? num_sms : 1);
   int best = 1;
   double best_fill = -1.0;
   for (int g = 1; g <= route_chunks(N); ++g) {
@@ -57,11 +54,14 @@ inline int route_launch_chunks(int64_t N, int row_blocks, int heads, int num_sms
   return best;
 }
 
+// Work buffer: a 256-byte status block (int32 status word first), the per-row errors, then the
+// per-chunk states.
+constexpr size_t kRouteStatusBytes = 256;
 size_t route_rowerr_bytes(int heads, int n_rows) {
   return ((size_t)heads * n_rows * 3 * sizeof(float) + 255) / 256 * 256;
 }
 size_t route_work_bytes(int heads, int64_t N, int d, int n_rows) {
-  return route_rowerr_bytes(heads, n_rows) +
+  return kRouteStatusBytes + route_rowerr_bytes(heads, n_rows) +
          (size_t)heads * n_rows * route_chunks(N) * 3 * (size_t)(d + 2) * sizeof(float);
 }
 
@@ -81,190 +81,370 @@ struct RouteParams {
   float* err;            // [H][2] nullable: relative errors of spatial / temporal
 };
 
-template <int D>
-struct RouteCfg {
-  static constexpr int KP = D + 8;   // padded bf16 K row: 16-byte reads of 8 consecutive lanes hit distinct banks
-  static constexpr int DPL = D / 32;
-  static constexpr size_t kQ = (size_t)kRouteRows * D * 4;
-  static constexpr size_t kP = (size_t)kRouteRows * kRouteKeys * 16;
-  static constexpr size_t kK = (size_t)kRouteKeys * KP * 2;
-  static constexpr size_t kV = (size_t)kRouteKeys * D * 2;
-  static constexpr size_t kBytes = kQ + kP + kK + kV + kRouteRows * 4;
-};
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
-  return x;
-}
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
   return x;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kRouteThreads, 2) route_partial_kernel(const RouteParams P) {
-  using C = RouteCfg<D>;
-  constexpr int DPL = C::DPL, KP = C::KP;
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* sQ = reinterpret_cast<float*>(smem);                                // [32][D], times sl2
-  float4* sP = reinterpret_cast<float4*>(smem + C::kQ);                      // [32][64] {dense, spatial, temporal, -}
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + C::kQ + C::kP);          // [64][KP]
-  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + C::kQ + C::kP + C::kK);  // [64][D]
-  int* sRow = reinterpret_cast<int*>(smem + C::kQ + C::kP + C::kK + C::kV);           // [32]
-  const int h = blockIdx.y, g = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j_begin = g * P.chunk;
-  const int j_end = min(P.N, j_begin + P.chunk);
-  if (tid < kRouteRows) {
-    const int idx = blockIdx.x * kRouteRows + tid;
-    int r = idx < P.n_rows ? P.rows[idx] : -1;
-    sRow[tid] = (r >= 0 && r < P.N) ? r : -1;  // rows outside the sequence attend with Q = 0, unused
-  }
-  __syncthreads();
-  const size_t hoff = (size_t)h * P.N * D;
-  for (int x = tid; x < kRouteRows * D; x += kRouteThreads) {
-    const int rr = x / D, c = x - rr * D, r = sRow[rr];
-    sQ[x] = r >= 0 ? __bfloat162float(P.q[hoff + (size_t)r * D + c]) * P.sl2 : 0.f;
-  }
-  const int S = P.gs.S;
-  int ti[4], si[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = max(sRow[4 * warp + i], 0);
-    ti[i] = r / S;
-    si[i] = r - ti[i] * S;
-  }
-  float m[4][3], l[4][3], o[4][3][DPL];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      m[i][a] = -INFINITY;
-      l[i][a] = 0.f;
-#pragma unroll
-      for (int x = 0; x < DPL; ++x) o[i][a][x] = 0.f;
-    }
+// ---------------------------------------------------------------------------------------
+// Tensor-core form. Sampled rows x keys is a contraction (S = Q_rows K^T, then three P V), so one
+// CTA takes up to 128 sampled rows of one head (M = 128; rows past the list are padding) and one
+// chunk of the keys, streamed in 64-key tiles by TMA:
+//   warps 0-3  one thread per row: load the row's Q into shared memory (128-byte swizzle), then per
+//              tile load S from TMEM, and for each mask (dense, spatial, temporal) update that
+//              mask's running maximum and sum, compute P = 2^(S sl2 - m) on its kept keys in fp32
+//              and store it into that mask's two P buffers in shared memory as a bf16 pair,
+//              P = P_hi + P_lo with P_hi = bf16(P), P_lo = bf16(P - P_hi) (about 16 significant
+//              bits, so that the route's error sums keep the fp32 path's accuracy);
+//   warp 4     TMA producer of the K / V ring;
+//   warp 5     MMA issuer: S(e) = Q K(e)^T into TMEM (N = 64), then O_a += P_hi,a V(e) + P_lo,a V(e)
+//              for the three masks into three TMEM accumulators. S(e + 1) is issued as soon as the softmax has
+//              loaded S(e) (P lives in shared memory), so it overlaps the softmax of tile e.
+// Every wait is bounded; the chunk state written out is the CUDA-core form's, so the same merge
+// and reduction kernels finish the route.
+constexpr int kRtRows = 128;
+constexpr int kRtKeys = kRouteKeys;
+constexpr int kRtStages = 4;
+constexpr int kRtThreads = 192;
+constexpr int kRtProducer = 4;
+constexpr int kRtMma = 5;
 
-  for (int j0 = j_begin; j0 < j_end; j0 += kRouteKeys) {
-    const int nt = min(kRouteKeys, j_end - j0);
-    __syncthreads();  // every warp is done with the previous tile
-    constexpr int CPR = D / 8;  // 16-byte pieces per row
-    for (int c = tid; c < kRouteKeys * CPR; c += kRouteThreads) {
-      const int key = c / CPR, part = c - key * CPR;
-      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
-      if (key < nt) {
-        const size_t off = hoff + (size_t)(j0 + key) * D + part * 8;
-        kv = __ldg(reinterpret_cast<const uint4*>(P.k + off));
-        vv = __ldg(reinterpret_cast<const uint4*>(P.v + off));
-      }
-      *reinterpret_cast<uint4*>(sK + key * KP + part * 8) = kv;
-      *reinterpret_cast<uint4*>(sV + key * D + part * 8) = vv;
+template <int D>
+struct RtCfg {
+  static constexpr int kChunks = D / 64;                   // 128-byte swizzle chunks per Q / K / V row
+  static constexpr int kQBytes = kRtRows * D * 2;
+  static constexpr int kPBytes = kRtRows * kRtKeys * 2;    // one P buffer: 128 rows x 128 bytes
+  static constexpr int kTileBytes = kRtKeys * D * 2;       // one K or V tile
+  static constexpr int kDataBytes = kQBytes + 6 * kPBytes + kRtStages * kTileBytes;  // P_hi, P_lo per mask
+  static constexpr int kSmemBytes = kDataBytes + 256 /*barriers*/ + 1024 /*alignment*/;
+  static constexpr uint32_t kSCol = 0;                     // S: 64 columns
+  __host__ __device__ static constexpr uint32_t o_col(int a) { return 128u + (uint32_t)D * a; }
+  static_assert(128 + 3 * D <= 512, "TMEM columns");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+struct RouteTcParams {
+  CUtensorMap tm_k, tm_v;  // [H, N, d] bf16 as (d, N, H), box 64 columns x 64 keys x 1 head
+  const __nv_bfloat16* q;
+  int H, N;
+  float sl2;
+  MaskGeom gs, gt;
+  const int32_t* rows;
+  int n_rows, G, chunk;
+  float* part;
+  int* status;
+};
+
+// barriers (8 bytes each): kv_full[NS], kv_empty[NS], q_full, s_full, s_free, p_ready, pv_done, drain
+struct RtBar {
+  uint32_t base;
+  __device__ uint32_t kv_full(uint32_t i) const { return base + 8u * i; }
+  __device__ uint32_t kv_empty(uint32_t i) const { return base + 8u * (kRtStages + i); }
+  __device__ uint32_t q_full() const { return base + 8u * (2 * kRtStages + 0); }
+  __device__ uint32_t s_full() const { return base + 8u * (2 * kRtStages + 1); }
+  __device__ uint32_t s_free() const { return base + 8u * (2 * kRtStages + 2); }
+  __device__ uint32_t p_ready() const { return base + 8u * (2 * kRtStages + 3); }
+  __device__ uint32_t pv_done() const { return base + 8u * (2 * kRtStages + 4); }
+  __device__ uint32_t drain() const { return base + 8u * (2 * kRtStages + 5); }
+  static constexpr int kCount = 2 * kRtStages + 6;
+  static constexpr uint32_t kAbortOff = 8u * kCount;       // abort flag
+  static constexpr uint32_t kTmemOff = kAbortOff + 8;      // TMEM base
+};
+
+// Keeps the kept keys' scores of one mask (bit j of keep) and folds them into the running state:
+// returns whether this thread's maximum grew past the rescale threshold (or had none yet).
+__device__ __forceinline__ bool rt_mask_max(const float* x, uint64_t keep, float m, float& m_new) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kRtKeys; ++j)
+    if ((keep >> j) & 1ull) mx = fmaxf(mx, x[j]);
+  m_new = fmaxf(m, mx);
+  return (m_new > m) && (m == -INFINITY || m_new - m > kRescaleLog2);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_constant__ RouteTcParams P) {
+  using C = RtCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sQ = sbase, sP = sQ + C::kQBytes, sRing = sP + 6 * C::kPBytes;
+  RtBar b;
+  b.base = sRing + kRtStages * C::kTileBytes;
+  uint8_t* ctl = smem_raw + (b.base - raw);
+  const uint32_t abort_addr = b.base + RtBar::kAbortOff;
+  int* status = P.status;
+  const int h = blockIdx.y, g = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j_begin = g * P.chunk, j_end = min(P.N, j_begin + P.chunk);
+  const int ntiles = (j_end - j_begin + kRtKeys - 1) / kRtKeys;
+
+  if (threadIdx.x == 0) {
+    uint64_t* bar = reinterpret_cast<uint64_t*>(ctl);
+    for (int i = 0; i < kRtStages; ++i) {
+      mbar_init(bar + i, 1);
+      mbar_init(bar + kRtStages + i, 1);
     }
-    __syncthreads();
-    // ---- scores of rows 4w..4w+3 with keys j0 + lane and j0 + lane + 32 (log2 units)
-    float sc[4][2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sc[i][0] = sc[i][1] = 0.f;
-#pragma unroll 4
-    for (int st = 0; st < D / 8; ++st) {
-      float fa[8], fb[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + lane * KP + st * 8), fa);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + (lane + 32) * KP + st * 8), fb);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 q0 = *reinterpret_cast<const float4*>(sQ + (4 * warp + i) * D + st * 8);
-        const float4 q1 = *reinterpret_cast<const float4*>(sQ + (4 * warp + i) * D + st * 8 + 4);
-        const float qq[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          sc[i][0] = fmaf(qq[x], fa[x], sc[i][0]);
-          sc[i][1] = fmaf(qq[x], fb[x], sc[i][1]);
+    mbar_init(bar + 2 * kRtStages + 0, kRtRows);  // q_full: every softmax thread wrote its Q row
+    mbar_init(bar + 2 * kRtStages + 1, 1);        // s_full
+    mbar_init(bar + 2 * kRtStages + 2, kRtRows);  // s_free
+    mbar_init(bar + 2 * kRtStages + 3, kRtRows);  // p_ready
+    mbar_init(bar + 2 * kRtStages + 4, 1);        // pv_done
+    mbar_init(bar + 2 * kRtStages + 5, 1);        // drain
+    *reinterpret_cast<volatile int*>(ctl + RtBar::kAbortOff) = 0;
+    fence_mbar_init();
+  }
+  if (warp == kRtMma) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(ctl + RtBar::kTmemOff), 512);
+    tmem_relinquish();
+  }
+  if (warp == kRtProducer && lane == 0) {
+    prefetch_tmap(&P.tm_k);
+    prefetch_tmap(&P.tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<uint32_t*>(ctl + RtBar::kTmemOff);
+
+  if (warp == kRtProducer) {
+    // ---------------------------------------------------------------- K / V tiles, in the order
+    // the MMA warp reads them: K(0), then K(e + 1), V(e) per tile
+    if (lane == 0) {
+      uint32_t pos = 0;
+      for (int n = 0; n < 2 * ntiles; ++n) {
+        int e, w;
+        if (n == 0) {
+          e = 0;
+          w = 0;
+        } else if (n == 2 * ntiles - 1) {
+          e = ntiles - 1;
+          w = 1;
+        } else {
+          const int m = n - 1;
+          e = (m >> 1) + ((m & 1) ^ 1);
+          w = m & 1;
+        }
+        const uint32_t st = pos % kRtStages;
+        if (!wait_bar(b.kv_empty(st), ((pos / kRtStages) & 1u) ^ 1u, abort_addr, status)) break;
+        mbar_expect_tx(b.kv_full(st), C::kTileBytes);
+        const uint32_t dst = sRing + st * C::kTileBytes;
+        for (int ch = 0; ch < C::kChunks; ++ch)
+          tma_load_3d(dst + ch * (kRtKeys * 128), w == 0 ? &P.tm_k : &P.tm_v, b.kv_full(st), ch * 64,
+                      j_begin + e * kRtKeys, h);
+        ++pos;
+      }
+      if (ld_shared_volatile(abort_addr)) {  // let issued copies land before the CTA may exit
+        const uint32_t n = pos < (uint32_t)kRtStages ? pos : (uint32_t)kRtStages;
+        for (uint32_t i = 0; i < n; ++i) {
+          const uint32_t q = pos - 1 - i;
+          drain_bar(b.kv_full(q % kRtStages), (q / kRtStages) & 1u);
         }
       }
-    }
-    // ---- masks and the three online softmaxes per row
-    const int ja = j0 + lane, jb = j0 + lane + 32;
-    const bool ina = lane < nt, inb = lane + 32 < nt;
-    const int tja = ja / S, sja = ja - tja * S, tjb = jb / S, sjb = jb - tjb * S;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool keep[3][2] = {
-          {ina, inb},
-          {ina && (tja < P.gs.F0 || abs(ti[i] - tja) <= P.gs.k), inb && (tjb < P.gs.F0 || abs(ti[i] - tjb) <= P.gs.k)},
-          {ina && (tja < P.gt.F0 || abs(si[i] - sja) <= P.gt.b), inb && (tjb < P.gt.F0 || abs(si[i] - sjb) <= P.gt.b)}};
-      float p[3][2];
-#pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        const float x0 = keep[a][0] ? sc[i][0] : -INFINITY;
-        const float x1 = keep[a][1] ? sc[i][1] : -INFINITY;
-        const float mn = fmaxf(m[i][a], warp_max(fmaxf(x0, x1)));
-        const float alpha = (mn == -INFINITY) ? 1.f : exp2f(m[i][a] - mn);
-        p[a][0] = keep[a][0] ? exp2f(x0 - mn) : 0.f;
-        p[a][1] = keep[a][1] ? exp2f(x1 - mn) : 0.f;
-        l[i][a] = l[i][a] * alpha + warp_sum(p[a][0] + p[a][1]);
-        m[i][a] = mn;
-#pragma unroll
-        for (int x = 0; x < DPL; ++x) o[i][a][x] *= alpha;
-      }
-      sP[(4 * warp + i) * kRouteKeys + lane] = make_float4(p[0][0], p[1][0], p[2][0], 0.f);
-      sP[(4 * warp + i) * kRouteKeys + lane + 32] = make_float4(p[0][1], p[1][1], p[2][1], 0.f);
     }
     __syncwarp();
-    // ---- O += P V over the tile's keys (P = 0 and V = 0 past the end)
-#pragma unroll 2
-    for (int jj = 0; jj < kRouteKeys; ++jj) {
-      float vv[DPL];
-      if constexpr (DPL == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(sV + jj * D + lane * DPL);
-        vv[0] = __uint_as_float(u.x << 16);
-        vv[1] = __uint_as_float(u.x & 0xffff0000u);
-        vv[2] = __uint_as_float(u.y << 16);
-        vv[3] = __uint_as_float(u.y & 0xffff0000u);
-      } else {
-        static_assert(DPL == 2, "head dim 64 or 128");
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(sV + jj * D + lane * DPL);
-        vv[0] = __uint_as_float(u << 16);
-        vv[1] = __uint_as_float(u & 0xffff0000u);
+  } else if (warp == kRtMma) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kRtKeys, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(D, true);
+      const uint64_t qdesc = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t kdesc = smem_desc_sw128(sRing, 16, 1024);
+      const uint64_t vdesc = smem_desc_sw128(sRing, kRtKeys * 128, 1024);
+      const uint64_t pdesc = smem_desc_sw128(sP, 16, 1024);
+      uint32_t pos = 0;
+      bool ok = wait_bar(b.q_full(), 0, abort_addr, status);
+      tc_fence_after();
+      auto issue_s = [&](uint32_t kpos) -> bool {
+        const uint32_t st = kpos % kRtStages;
+        if (!wait_bar(b.kv_full(st), (kpos / kRtStages) & 1u, abort_addr, status)) return false;
+        const uint64_t kd = kdesc + ((st * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qoff = ((kk >> 2) * (kRtRows * 128) + (kk & 3) * 32) >> 4;
+          const uint32_t koff = ((kk >> 2) * (kRtKeys * 128) + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + C::kSCol, qdesc + qoff, kd + koff, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(b.s_full());
+        umma_commit(b.kv_empty(st));
+        return true;
+      };
+      if (ok && ntiles > 0) ok = issue_s(pos++);
+      for (int e = 0; e < ntiles && ok; ++e) {
+        if (e + 1 < ntiles) {  // S(e + 1) once the softmax has loaded S(e)
+          ok = wait_bar(b.s_free(), (uint32_t)e & 1u, abort_addr, status);
+          if (!ok) break;
+          tc_fence_after();
+          ok = issue_s(pos++);
+          if (!ok) break;
+        }
+        const uint32_t vpos = pos++;
+        const uint32_t st = vpos % kRtStages;
+        ok = wait_bar(b.p_ready(), (uint32_t)e & 1u, abort_addr, status) &&
+             wait_bar(b.kv_full(st), (vpos / kRtStages) & 1u, abort_addr, status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t vd = vdesc + ((st * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {  // buffer 2a: P_hi, 2a + 1: P_lo
+            const uint64_t pd = pdesc + (((2 * a + part) * C::kPBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kRtKeys / 16; ++kk)
+              umma_ss(tmem + C::o_col(a), pd + (((kk & 3) * 32) >> 4), vd + ((kk * 2048) >> 4), idesc_o,
+                      (e > 0 || part > 0 || kk > 0) ? 1u : 0u);
+          }
+        umma_commit(b.pv_done());
+        umma_commit(b.kv_empty(st));
       }
+      umma_commit(b.drain());
+      drain_bar(b.drain(), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- rows: Q, softmaxes, state out
+    const int lr = threadIdx.x;  // row within the block = TMEM lane
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int ridx = blockIdx.x * kRtRows + lr;
+    int r = ridx < P.n_rows ? __ldg(P.rows + ridx) : -1;
+    if (r < 0 || r >= P.N) r = 0;  // padding and rows outside the sequence: any valid row, unused
+    const int S = P.gs.S;
+    const int ti = r / S, si = r - ti * S;
+    {  // Q row into the 128-byte-swizzle K-major tile: chunk c, row lr, 16-byte unit u at u ^ (lr % 8)
+      const uint4* src = reinterpret_cast<const uint4*>(P.q + ((size_t)h * P.N + r) * D);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 pp = sP[(4 * warp + i) * kRouteKeys + jj];
+      for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
-        for (int x = 0; x < DPL; ++x) {
-          o[i][0][x] = fmaf(pp.x, vv[x], o[i][0][x]);
-          o[i][1][x] = fmaf(pp.y, vv[x], o[i][1][x]);
-          o[i][2][x] = fmaf(pp.z, vv[x], o[i][2][x]);
+        for (uint32_t u = 0; u < 8; ++u) {
+          const uint4 v = __ldg(src + c * 8 + u);
+          st_shared_v4(sQ + c * (kRtRows * 128) + (uint32_t)lr * 128u + ((u ^ ((uint32_t)lr & 7u)) << 4), v.x, v.y,
+                       v.z, v.w);
+        }
+      fence_proxy_async_shared();
+      mbar_arrive(b.q_full());
+    }
+    float m[3] = {-INFINITY, -INFINITY, -INFINITY}, l[3] = {0.f, 0.f, 0.f};
+    bool ok = true;
+    for (int e = 0; e < ntiles; ++e) {
+      if (!__all_sync(0xffffffffu, wait_bar(b.s_full(), (uint32_t)e & 1u, abort_addr, status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[kRtKeys];
+      tmem_ld32(tmem + lane_off + C::kSCol, sr);
+      tmem_ld32(tmem + lane_off + C::kSCol + 32, sr + 32);
+      tmem_ld_wait();
+      tmem_ld_fence32(sr);
+      tmem_ld_fence32(sr + 32);
+      tc_fence_before();
+      mbar_arrive(b.s_free());
+      float x[kRtKeys];
+#pragma unroll
+      for (int j = 0; j < kRtKeys; ++j) x[j] = __uint_as_float(sr[j]) * P.sl2;
+      // kept keys of each mask in this tile (original identities, key j = t * S + s)
+      const int j0 = j_begin + e * kRtKeys;
+      int tj = j0 / S, sj = j0 - tj * S;
+      uint64_t keep[3] = {0ull, 0ull, 0ull};
+#pragma unroll
+      for (int j = 0; j < kRtKeys; ++j) {
+        const bool in = j0 + j < j_end;
+        const bool sink = tj < P.gs.F0;
+        keep[0] |= (uint64_t)in << j;
+        keep[1] |= (uint64_t)(in && (sink || abs(ti - tj) <= P.gs.k)) << j;
+        keep[2] |= (uint64_t)(in && (sink || abs(si - sj) <= P.gt.b)) << j;
+        if (++sj == S) {
+          sj = 0;
+          ++tj;
         }
       }
+      // the previous tile's P V are complete: the P buffers are free and O holds them
+      if (e > 0 && !__all_sync(0xffffffffu, wait_bar(b.pv_done(), (uint32_t)(e - 1) & 1u, abort_addr, status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        float mn;
+        const bool need = rt_mask_max(x, keep[a], m[a], mn);
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = (mn == -INFINITY) ? 1.f : ex2f(m[a] - mn);
+          l[a] *= alpha;
+          m[a] = mn;
+          if (e > 0) {  // O_a holds the earlier tiles' P V (tile 0's MMA overwrites it)
+            const uint32_t tO = tmem + lane_off + C::o_col(a);
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+              uint32_t o[32];
+              tmem_ld32(tO + q * 32, o);
+              tmem_ld_wait();
+              tmem_ld_fence32(o);
+#pragma unroll
+              for (int y = 0; y < 32; ++y) o[y] = __float_as_uint(__uint_as_float(o[y]) * alpha);
+              tmem_st32(tO + q * 32, o);
+            }
+            tmem_st_wait();
+          }
+        }
+        uint32_t hi[kRtKeys / 2], lo[kRtKeys / 2];
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < kRtKeys; j += 2) {
+          const float p0 = ((keep[a] >> j) & 1ull) ? ex2f(x[j] - m[a]) : 0.f;
+          const float p1 = ((keep[a] >> (j + 1)) & 1ull) ? ex2f(x[j + 1] - m[a]) : 0.f;
+          sum += p0 + p1;
+          hi[j / 2] = pack_bf16(p0, p1);
+          const float h0 = __uint_as_float(hi[j / 2] << 16), h1 = __uint_as_float(hi[j / 2] & 0xFFFF0000u);
+          lo[j / 2] = pack_bf16(p0 - h0, p1 - h1);
+        }
+        l[a] += sum;
+        store_p_sw128<kRtKeys>(sP + (2 * a) * C::kPBytes, lr, hi);
+        store_p_sw128<kRtKeys>(sP + (2 * a + 1) * C::kPBytes, lr, lo);
+      }
+      fence_proxy_async_shared();
+      tc_fence_before();
+      mbar_arrive(b.p_ready());
     }
-  }
-  // ---- this chunk's state of every row the block holds
+    // ---- this chunk's state of the row: O (unnormalised), running max (log2 units), sum
+    if (ok && ntiles > 0 && __all_sync(0xffffffffu, wait_bar(b.pv_done(), (uint32_t)(ntiles - 1) & 1u, abort_addr,
+                                                            status))) {
+      tc_fence_after();
+      const bool write = ridx < P.n_rows;
+      float* dst = P.part + (((size_t)h * P.n_rows + (write ? ridx : 0)) * P.G + g) * 3 * (D + 2);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int ridx = blockIdx.x * kRouteRows + 4 * warp + i;
-    if (ridx >= P.n_rows) continue;
-    float* dst = P.part + (((size_t)h * P.n_rows + ridx) * P.G + g) * 3 * (D + 2);
+      for (int a = 0; a < 3; ++a) {
+#pragma unroll 1
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + C::o_col(a) + q * 32, o);
+          tmem_ld_wait();
+          tmem_ld_fence32(o);
+          if (write) {  // (a row's state is 4-byte aligned only: scalar stores)
 #pragma unroll
-    for (int a = 0; a < 3; ++a) {
-#pragma unroll
-      for (int x = 0; x < DPL; ++x) dst[a * (D + 2) + lane * DPL + x] = o[i][a][x];
-      if (lane == 0) {
-        dst[a * (D + 2) + D] = m[i][a];
-        dst[a * (D + 2) + D + 1] = l[i][a];
+            for (int y = 0; y < 32; ++y) dst[a * (D + 2) + q * 32 + y] = __uint_as_float(o[y]);
+          }
+        }
+        if (write) {
+          dst[a * (D + 2) + D] = m[a];
+          dst[a * (D + 2) + D + 1] = l[a];
+        }
+      }
+    } else if (ntiles == 0 && ridx < P.n_rows) {  // an empty chunk: nothing kept
+      float* dst = P.part + (((size_t)h * P.n_rows + ridx) * P.G + g) * 3 * (D + 2);
+      for (int a = 0; a < 3; ++a) {
+        for (int y = 0; y < D; ++y) dst[a * (D + 2) + y] = 0.f;
+        dst[a * (D + 2) + D] = -INFINITY;
+        dst[a * (D + 2) + D + 1] = 0.f;
       }
     }
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kRtMma) tmem_dealloc(tmem, 512);
 }
 
 // One warp per (sampled row, head): combine the chunks' states of each mask, then the row's
@@ -337,22 +517,20 @@ __global__ void route_reduce_kernel(const RouteParams P) {
 }
 
 template <int D>
-static cudaError_t launch_partial(const RouteParams& P, int nblk_rows, int nchunks, cudaStream_t st) {
-  using C = RouteCfg<D>;
-  auto kern = route_partial_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kBytes);
+static cudaError_t launch_tc(const RouteTcParams& T, int nblk_rows, cudaStream_t st) {
+  using C = RtCfg<D>;
+  auto kern = route_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(nblk_rows, P.H, nchunks), kRouteThreads, C::kBytes, st>>>(P);
+  kern<<<dim3(nblk_rows, T.H, T.G), kRtThreads, C::kSmemBytes, st>>>(T);
   return cudaGetLastError();
 }
 
-int launch_route(const void* q, const void* k, const void* v, int heads, int N, int d, float scale, svg_geom geom,
-                 svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
+int launch_route(const void* q, const CUtensorMap* tm_k, const CUtensorMap* tm_v, int heads, int N, int d, float scale,
+                 svg_geom geom, svg_mask mask, const int32_t* rows, int n_rows, void* work, uint8_t* route, float* err,
                  int num_sms, cudaStream_t st) {
   RouteParams P;
-  P.q = static_cast<const __nv_bfloat16*>(q);
-  P.k = static_cast<const __nv_bfloat16*>(k);
-  P.v = static_cast<const __nv_bfloat16*>(v);
+  memset(&P, 0, sizeof(P));
   P.H = heads;
   P.N = N;
   P.D = d;
@@ -361,15 +539,34 @@ int launch_route(const void* q, const void* k, const void* v, int heads, int N, 
   P.gt = make_geom(geom, mask, SVG_ROUTE_TEMPORAL);
   P.rows = rows;
   P.n_rows = n_rows;
-  const int nblk_rows = (n_rows + kRouteRows - 1) / kRouteRows;
-  P.chunk = route_chunk_len(N, route_launch_chunks(N, nblk_rows, heads, num_sms));
+  const int nblk_rows = (n_rows + kRtRows - 1) / kRtRows;
+  P.chunk = route_chunk_len(N, route_launch_chunks(N, nblk_rows, heads, num_sms, 1));
   P.G = (N + P.chunk - 1) / P.chunk;  // non-empty chunks, at most route_chunks(N)
-  P.rowerr = static_cast<float*>(work);
-  P.part = reinterpret_cast<float*>(static_cast<unsigned char*>(work) + route_rowerr_bytes(heads, n_rows));
+  unsigned char* wb = static_cast<unsigned char*>(work);
+  P.rowerr = reinterpret_cast<float*>(wb + kRouteStatusBytes);
+  P.part = reinterpret_cast<float*>(wb + kRouteStatusBytes + route_rowerr_bytes(heads, n_rows));
   P.route = route;
   P.err = err;
-  cudaError_t e = d == 128 ? launch_partial<128>(P, nblk_rows, P.G, st) : launch_partial<64>(P, nblk_rows, P.G, st);
-  if (e != cudaSuccess) return record_cuda_error("launch route_partial_kernel", e);
+  RouteTcParams T;
+  memset(&T, 0, sizeof(T));
+  T.tm_k = *tm_k;
+  T.tm_v = *tm_v;
+  T.q = static_cast<const __nv_bfloat16*>(q);
+  T.H = heads;
+  T.N = N;
+  T.sl2 = P.sl2;
+  T.gs = P.gs;
+  T.gt = P.gt;
+  T.rows = rows;
+  T.n_rows = n_rows;
+  T.G = P.G;
+  T.chunk = P.chunk;
+  T.part = P.part;
+  T.status = reinterpret_cast<int*>(wb);
+  cudaError_t e = cudaMemsetAsync(wb, 0, sizeof(int), st);
+  if (e != cudaSuccess) return record_cuda_error("cudaMemsetAsync(route status)", e);
+  e = d == 128 ? launch_tc<128>(T, nblk_rows, st) : launch_tc<64>(T, nblk_rows, st);
+  if (e != cudaSuccess) return record_cuda_error("launch route_tc_kernel", e);
   route_merge_kernel<<<dim3(n_rows, heads), 32, 0, st>>>(P);
   route_reduce_kernel<<<(heads + 127) / 128, 128, 0, st>>>(P);
   e = cudaGetLastError();

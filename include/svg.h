@@ -262,14 +262,18 @@ int svg_attention_fwd_noalloc(const void *q, const void *k, const void *v, void 
  * the spatial or the temporal mask based on sampled rows ("Sparse Attention Patterns"; summary of
  * the case study). For every head, the query rows listed in d_rows (ORIGINAL token indices,
  * frame-major) attend to all keys under the dense mask, the spatial mask and the temporal mask of
- * `mask` (exact variant, original token order; layout and variant are ignored), in fp32. With
- * E_m = sum over the rows of |O_m - O_dense|^2 and E_d = sum of |O_dense|^2:
+ * `mask` (exact variant, original token order; layout and variant are ignored): scores and the
+ * three P V products on the tensor cores (bf16 operands, fp32 accumulation; P rounded to bf16 as in
+ * the attention kernel), one online softmax per mask in fp32. With E_m = sum over the rows of
+ * |O_m - O_dense|^2 and E_d = sum of |O_dense|^2:
  *   d_route[h] = E_spatial <= E_temporal ? SVG_ROUTE_SPATIAL : SVG_ROUTE_TEMPORAL
  *   d_err[2h], d_err[2h+1] = E_spatial / E_d, E_temporal / E_d   (d_err nullable)
  *   q, k, v:  [heads, tokens, d] bf16 in ORIGINAL order (before any permutation).
  *   d_rows:   device int32 [n_rows]; entries outside [0, tokens) are ignored.
- *   d_work:   device buffer of svg_route_work_bytes(heads, tokens, d, n_rows) bytes, 4-byte
- *             aligned (per-row errors, and the softmax state of each key chunk of each row).
+ *   d_work:   device buffer of svg_route_work_bytes(heads, tokens, d, n_rows) bytes, 256-byte
+ *             aligned: a device status word first (0, or SVG_ERR_TIMEOUT when a pipeline wait ran
+ *             out; svg_read_status(d_work) reads it), then the per-row errors and the softmax
+ *             state of each key chunk of each row.
  *   d_route:  device uint8 [heads].
  * The sums over rows run in a fixed order, so the decision is deterministic.
  * Errors: SVG_ERR_ARG (null or misaligned pointer, bad geometry/mask, tokens != frames*H*W),

@@ -126,10 +126,10 @@ def test_route_argument_checks(svg):
     g, m = svg.make_geom(4, 8, 16), svg.make_mask(1, 16)
     wb = svg.svg_route_work_bytes
     assert wb(2, 512, 64, 0) == 0 and wb(0, 512, 64, 8) == 0 and wb(2, 512, 96, 8) == 0
-    # per-row errors (rounded to 256 bytes) + one chunk state of 3 x (d + 2) floats per row
-    assert wb(2, 512, 64, 8) == 256 + 2 * 8 * 1 * 3 * 66 * 4
+    # status block + per-row errors (rounded to 256 bytes) + one chunk state of 3 x (d + 2) floats per row
+    assert wb(2, 512, 64, 8) == 256 + 256 + 2 * 8 * 1 * 3 * 66 * 4
     # 75,600 keys: 37 chunks of 2,048 would exceed the cap of 32
-    assert wb(10, 75600, 128, 64) == (10 * 64 * 3 * 4 + 255) // 256 * 256 + 10 * 64 * 32 * 3 * 130 * 4
+    assert wb(10, 75600, 128, 64) == 256 + (10 * 64 * 3 * 4 + 255) // 256 * 256 + 10 * 64 * 32 * 3 * 130 * 4
     f = lib.svg_route_heads
     f.argtypes = svg._sig["svg_route_heads"][1]
     p, rt = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 24)
@@ -139,6 +139,8 @@ def test_route_argument_checks(svg):
     assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 8, p, ok_bytes, None, None, None) == -1        # null route
     assert f(ctypes.c_void_p((1 << 20) + 8), p, p, 2, 512, 64, 0.0, g, m, p, 8, p, ok_bytes, rt, None,
              None) == -1                                                                    # misaligned q
+    assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 8, ctypes.c_void_p((1 << 20) + 64), ok_bytes, rt, None,
+             None) == -1                                                                    # misaligned work
     assert f(p, p, p, 2, 511, 64, 0.0, g, m, p, 8, p, ok_bytes, rt, None, None) == -1         # tokens mismatch
     assert f(p, p, p, 2, 512, 64, 0.0, g, m, p, 0, p, ok_bytes, rt, None, None) == -1         # no rows
     assert f(p, p, p, 2, 512, 96, 0.0, g, m, p, 8, p, ok_bytes, rt, None, None) == -2         # d

@@ -359,8 +359,10 @@ def _route_case(S, w, q, k, v, rows):
     rd = torch.as_tensor(np.asarray(rows), dtype=torch.int32, device=dev)
     route = torch.full((w.heads,), 255, dtype=torch.uint8, device=dev)
     err = torch.full((w.heads, 2), -1.0, dtype=torch.float32, device=dev)
-    S.svg_route_heads(qd, kd, vd, g, m, rd, route, err)
+    work = torch.empty(S.svg_route_work_bytes(w.heads, w.tokens, w.d, len(rows)), dtype=torch.uint8, device=dev)
+    S.svg_route_heads(qd, kd, vd, g, m, rd, route, err, work=work)
     torch.cuda.synchronize()
+    assert S.svg_read_status(work) == 0
     valid = [r for r in np.asarray(rows).tolist() if 0 <= r < w.tokens]
     want_err, want_route = [], []
     for h in range(w.heads):
@@ -413,6 +415,17 @@ def test_route_pages_shape(S):
     got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
     _check_routes(got_r, got_e, want_r, want_e)
     assert list(got_r) == kinds
+
+
+def test_route_many_rows_several_row_blocks(S):
+    """300 sampled rows per head: three 128-row blocks of the tensor-core kernel, the last ragged."""
+    w = syn.Workload("route_rows", frames=6, grid_h=10, grid_w=16, routes=(0, 1), d=128, frame_window=1,
+                     spatial_band=12)
+    q, k, v = syn.make_routed_qkv(w, list(w.routes), strength=1.2, seed_offset=5)
+    rows = np.sort(np.random.default_rng(3).choice(w.tokens, 300, replace=False))
+    got_r, got_e, want_r, want_e = _route_case(S, w, q, k, v, rows)
+    _check_routes(got_r, got_e, want_r, want_e)
+    assert list(got_r) == list(w.routes)
 
 
 @pytest.mark.parametrize("d", [64, 128])
