@@ -242,6 +242,9 @@ def main():
                     help="split one call's heads over the ranks (strong scaling) instead of running replicas")
     ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=96, help="oracle rows per head per --impl reference step")
+    ap.add_argument("--route-calls", type=int, default=0,
+                    help="after the timed region, this many svg_route_heads calls (64 sampled rows per head) on the "
+                         "workload, untimed: a fixed launch sequence for profiling the route kernel")
     ap.add_argument("--clock-log-dir", default="",
                     help="folder for the nvidia-smi clock samples of the timed region (default: the temp folder)")
     args = ap.parse_args()
@@ -341,6 +344,18 @@ def main():
                 "frac": achieved / peak, "traffic": captured_traffic(w, args),
                 "kernel": f"attn_kernel<128,128> ({args.mode}, {kernel_variant()} schedule)",
                 "flop_definition": "4*d*(in-range area of visited tiles)", "peak_kind": f"{peak_kind} bf16 burst"}
+
+    if args.route_calls > 0:
+        rrows = torch.as_tensor(syn.sample_rows(w.replace(sample_rows=64), 0)[:64].numpy(), dtype=torch.int32,
+                                device=dev)
+        rt = torch.empty(w.heads, dtype=torch.uint8, device=dev)
+        rwork = torch.empty(S.svg_route_work_bytes(w.heads, w.tokens, w.d, rrows.numel()), dtype=torch.uint8,
+                            device=dev)
+        for _ in range(args.route_calls):
+            S.svg_route_heads(q, k, v, g, m, rrows, rt, work=rwork)
+        torch.cuda.synchronize()
+        if S.svg_read_status(rwork) != 0:
+            raise RuntimeError("route kernel status")
 
     extras = {}
     if not (args.no_extras or args.quick):
@@ -478,6 +493,14 @@ def side_measurements(S, w, g, m, t, routes, q, k, v, qp, kp, vp, o, scratch, ws
     work = torch.empty(S.svg_route_work_bytes(w.heads, w.tokens, w.d, rows.numel()), dtype=torch.uint8, device=dev)
     out["route_ms"] = time_events(lambda: S.svg_route_heads(q, k, v, g, m, rows, rt, work=work), 5, stream)
     out["route_rows_per_head"] = int(rows.numel())
+    rows256 = torch.as_tensor(syn.sample_rows(w.replace(sample_rows=256), 0)[:256].numpy(), dtype=torch.int32,
+                              device=dev)
+    work256 = torch.empty(S.svg_route_work_bytes(w.heads, w.tokens, w.d, rows256.numel()), dtype=torch.uint8,
+                          device=dev)
+    out["route_ms_256_rows"] = time_events(lambda: S.svg_route_heads(q, k, v, g, m, rows256, rt, work=work256), 5,
+                                           stream)
+    out["route_status"] = S.svg_read_status(work256)
+    del work256
     out["scheduler"] = scheduler_compare(S, w, qp, kp, vp, o, routes, ws, g, m, t, scratch, stream, dev)
     out["workloads"] = other_workloads(S, P, stream, dev)
     out["tile_sweep_mixed_75600"] = tile_sweep(S, stream, dev)

@@ -136,7 +136,9 @@ struct RouteTcParams {
   int* status;
 };
 
-// barriers (8 bytes each): kv_full[NS], kv_empty[NS], q_full, s_full, s_free, p_ready, pv_done, drain
+// barriers (8 bytes each): kv_full[NS], kv_empty[NS], q_full, s_full, s_free, p_ready[3], pv_done[3],
+// drain -- one p_ready / pv_done per mask, so that each mask's P store waits only for that mask's
+// previous P V
 struct RtBar {
   uint32_t base;
   __device__ uint32_t kv_full(uint32_t i) const { return base + 8u * i; }
@@ -144,13 +146,21 @@ struct RtBar {
   __device__ uint32_t q_full() const { return base + 8u * (2 * kRtStages + 0); }
   __device__ uint32_t s_full() const { return base + 8u * (2 * kRtStages + 1); }
   __device__ uint32_t s_free() const { return base + 8u * (2 * kRtStages + 2); }
-  __device__ uint32_t p_ready() const { return base + 8u * (2 * kRtStages + 3); }
-  __device__ uint32_t pv_done() const { return base + 8u * (2 * kRtStages + 4); }
-  __device__ uint32_t drain() const { return base + 8u * (2 * kRtStages + 5); }
-  static constexpr int kCount = 2 * kRtStages + 6;
+  __device__ uint32_t p_ready(int a) const { return base + 8u * (2 * kRtStages + 3 + a); }
+  __device__ uint32_t pv_done(int a) const { return base + 8u * (2 * kRtStages + 6 + a); }
+  __device__ uint32_t drain() const { return base + 8u * (2 * kRtStages + 9); }
+  static constexpr int kCount = 2 * kRtStages + 10;
   static constexpr uint32_t kAbortOff = 8u * kCount;       // abort flag
   static constexpr uint32_t kTmemOff = kAbortOff + 8;      // TMEM base
 };
+
+// Bits [lo - j0, hi - j0) of a 64-key tile starting at key j0 (clamped to the tile).
+__device__ __forceinline__ uint64_t rt_range_bits(int j0, int lo, int hi) {
+  const int a = max(lo - j0, 0), b = min(hi - j0, kRtKeys);
+  if (b <= a) return 0ull;
+  const uint64_t upto_b = b >= 64 ? ~0ull : ((1ull << b) - 1ull);
+  return upto_b & ~((1ull << a) - 1ull);
+}
 
 // Keeps the kept keys' scores of one mask (bit j of keep) and folds them into the running state:
 // returns whether this thread's maximum grew past the rescale threshold (or had none yet).
@@ -189,9 +199,11 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
     mbar_init(bar + 2 * kRtStages + 0, kRtRows);  // q_full: every softmax thread wrote its Q row
     mbar_init(bar + 2 * kRtStages + 1, 1);        // s_full
     mbar_init(bar + 2 * kRtStages + 2, kRtRows);  // s_free
-    mbar_init(bar + 2 * kRtStages + 3, kRtRows);  // p_ready
-    mbar_init(bar + 2 * kRtStages + 4, 1);        // pv_done
-    mbar_init(bar + 2 * kRtStages + 5, 1);        // drain
+    for (int a = 0; a < 3; ++a) {
+      mbar_init(bar + 2 * kRtStages + 3 + a, kRtRows);  // p_ready[a]
+      mbar_init(bar + 2 * kRtStages + 6 + a, 1);        // pv_done[a]
+    }
+    mbar_init(bar + 2 * kRtStages + 9, 1);  // drain
     *reinterpret_cast<volatile int*>(ctl + RtBar::kAbortOff) = 0;
     fence_mbar_init();
   }
@@ -281,13 +293,13 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
         }
         const uint32_t vpos = pos++;
         const uint32_t st = vpos % kRtStages;
-        ok = wait_bar(b.p_ready(), (uint32_t)e & 1u, abort_addr, status) &&
-             wait_bar(b.kv_full(st), (vpos / kRtStages) & 1u, abort_addr, status);
-        if (!ok) break;
-        tc_fence_after();
+        ok = wait_bar(b.kv_full(st), (vpos / kRtStages) & 1u, abort_addr, status);
         const uint64_t vd = vdesc + ((st * C::kTileBytes) >> 4);
 #pragma unroll
-        for (int a = 0; a < 3; ++a)
+        for (int a = 0; a < 3 && ok; ++a) {  // each mask's P V as soon as its P is stored
+          ok = wait_bar(b.p_ready(a), (uint32_t)e & 1u, abort_addr, status);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
           for (int part = 0; part < 2; ++part) {  // buffer 2a: P_hi, 2a + 1: P_lo
             const uint64_t pd = pdesc + (((2 * a + part) * C::kPBytes) >> 4);
@@ -296,7 +308,9 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
               umma_ss(tmem + C::o_col(a), pd + (((kk & 3) * 32) >> 4), vd + ((kk * 2048) >> 4), idesc_o,
                       (e > 0 || part > 0 || kk > 0) ? 1u : 0u);
           }
-        umma_commit(b.pv_done());
+          umma_commit(b.pv_done(a));
+        }
+        if (!ok) break;
         umma_commit(b.kv_empty(st));
       }
       umma_commit(b.drain());
@@ -344,36 +358,51 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
       float x[kRtKeys];
 #pragma unroll
       for (int j = 0; j < kRtKeys; ++j) x[j] = __uint_as_float(sr[j]) * P.sl2;
-      // kept keys of each mask in this tile (original identities, key j = t * S + s)
+      // kept keys of each mask in this tile, as bit sets from their ranges of original key index
+      // (key j = t * S + s): dense [j0, j_end); sink [0, F0 * S); spatial frames [ti - k, ti + k];
+      // temporal, in every frame t the tile touches, patches [si - b, si + b]
       const int j0 = j_begin + e * kRtKeys;
-      int tj = j0 / S, sj = j0 - tj * S;
-      uint64_t keep[3] = {0ull, 0ull, 0ull};
-#pragma unroll
-      for (int j = 0; j < kRtKeys; ++j) {
-        const bool in = j0 + j < j_end;
-        const bool sink = tj < P.gs.F0;
-        keep[0] |= (uint64_t)in << j;
-        keep[1] |= (uint64_t)(in && (sink || abs(ti - tj) <= P.gs.k)) << j;
-        keep[2] |= (uint64_t)(in && (sink || abs(si - sj) <= P.gt.b)) << j;
-        if (++sj == S) {
-          sj = 0;
-          ++tj;
-        }
+      const int jl = min(j0 + kRtKeys, j_end);  // end of this tile's keys
+      uint64_t keep[3];
+      keep[0] = rt_range_bits(j0, j0, jl);
+      const uint64_t sink = rt_range_bits(j0, 0, P.gs.F0 * S) & keep[0];
+      keep[1] = (rt_range_bits(j0, max(ti - P.gs.k, 0) * S, (min(ti + P.gs.k, P.gs.T - 1) + 1) * S) & keep[0]) | sink;
+      {
+        const int s0 = max(si - P.gt.b, 0), s1 = min(si + P.gt.b, S - 1) + 1;
+        uint64_t band = 0ull;
+        for (int t = j0 / S; t * S < jl; ++t) band |= rt_range_bits(j0, t * S + s0, t * S + s1);
+        keep[2] = (band & keep[0]) | sink;
       }
-      // the previous tile's P V are complete: the P buffers are free and O holds them
-      if (e > 0 && !__all_sync(0xffffffffu, wait_bar(b.pv_done(), (uint32_t)(e - 1) & 1u, abort_addr, status))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
         float mn;
         const bool need = rt_mask_max(x, keep[a], m[a], mn);
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = (mn == -INFINITY) ? 1.f : ex2f(m[a] - mn);
+        const bool rescale = __any_sync(0xffffffffu, need);
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = (mn == -INFINITY) ? 1.f : ex2f(m[a] - mn);
           l[a] *= alpha;
           m[a] = mn;
+        }
+        uint32_t hi[kRtKeys / 2], lo[kRtKeys / 2];
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < kRtKeys; j += 2) {
+          const float p0 = ((keep[a] >> j) & 1ull) ? ex2f(x[j] - m[a]) : 0.f;
+          const float p1 = ((keep[a] >> (j + 1)) & 1ull) ? ex2f(x[j + 1] - m[a]) : 0.f;
+          sum += p0 + p1;
+          hi[j / 2] = pack_bf16(p0, p1);
+          const float h0 = __uint_as_float(hi[j / 2] << 16), h1 = __uint_as_float(hi[j / 2] & 0xFFFF0000u);
+          lo[j / 2] = pack_bf16(p0 - h0, p1 - h1);
+        }
+        l[a] += sum;
+        // this mask's previous P V is complete: its P buffers are free and O_a holds it
+        if (e > 0 && !__all_sync(0xffffffffu, wait_bar(b.pv_done(a), (uint32_t)(e - 1) & 1u, abort_addr, status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (rescale) {
           if (e > 0) {  // O_a holds the earlier tiles' P V (tile 0's MMA overwrites it)
             const uint32_t tO = tmem + lane_off + C::o_col(a);
 #pragma unroll 1
@@ -389,28 +418,20 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
             tmem_st_wait();
           }
         }
-        uint32_t hi[kRtKeys / 2], lo[kRtKeys / 2];
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < kRtKeys; j += 2) {
-          const float p0 = ((keep[a] >> j) & 1ull) ? ex2f(x[j] - m[a]) : 0.f;
-          const float p1 = ((keep[a] >> (j + 1)) & 1ull) ? ex2f(x[j + 1] - m[a]) : 0.f;
-          sum += p0 + p1;
-          hi[j / 2] = pack_bf16(p0, p1);
-          const float h0 = __uint_as_float(hi[j / 2] << 16), h1 = __uint_as_float(hi[j / 2] & 0xFFFF0000u);
-          lo[j / 2] = pack_bf16(p0 - h0, p1 - h1);
-        }
-        l[a] += sum;
         store_p_sw128<kRtKeys>(sP + (2 * a) * C::kPBytes, lr, hi);
         store_p_sw128<kRtKeys>(sP + (2 * a + 1) * C::kPBytes, lr, lo);
+        fence_proxy_async_shared();
+        tc_fence_before();
+        mbar_arrive(b.p_ready(a));
       }
-      fence_proxy_async_shared();
-      tc_fence_before();
-      mbar_arrive(b.p_ready());
+      if (!ok) break;
     }
     // ---- this chunk's state of the row: O (unnormalised), running max (log2 units), sum
-    if (ok && ntiles > 0 && __all_sync(0xffffffffu, wait_bar(b.pv_done(), (uint32_t)(ntiles - 1) & 1u, abort_addr,
-                                                            status))) {
+    bool done = ok && ntiles > 0;
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+      done = done && __all_sync(0xffffffffu, wait_bar(b.pv_done(a), (uint32_t)(ntiles - 1) & 1u, abort_addr, status));
+    if (done) {
       tc_fence_after();
       const bool write = ridx < P.n_rows;
       float* dst = P.part + (((size_t)h * P.n_rows + (write ? ridx : 0)) * P.G + g) * 3 * (D + 2);
