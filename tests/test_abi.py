@@ -207,3 +207,19 @@ def test_stall_test_entry_checks_arguments_like_the_regular_call(svg):
     p = ctypes.c_void_p(1 << 20)
     assert f(None, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -1
     assert f(p, p, p, p, None, 2, 512, 96, 0.0, routes, p, p, g, m, t, 0, p, 256, None, None) == -2
+
+
+def test_extended_entry_argument_checks(svg):
+    """svg_attention_fwd_ex: a missing options struct, an unknown order and a trace buffer without
+    entries or misaligned are rejected before any device work."""
+    lib = ctypes.CDLL(svg.LIB_PATH)
+    f = lib.svg_attention_fwd_ex
+    f.argtypes = svg._sig["svg_attention_fwd_ex"][1]
+    g, m, t = svg.make_geom(4, 8, 16), svg.make_mask(1, 16), svg.make_tile(64, 64)
+    routes = (ctypes.c_uint8 * 2)(0, 1)
+    p = ctypes.c_void_p(1 << 20)
+    args = (p, p, p, p, None, 2, 512, 64, 0.0, routes, p, p, g, m, t, 0, p, 256, None)
+    assert f(*args, None, None) == -1
+    assert f(*args, ctypes.byref(svg.svg_launch_opts(7, None, 0)), None) == -1
+    assert f(*args, ctypes.byref(svg.svg_launch_opts(svg.SVG_ORDER_WORK, (1 << 20), 0)), None) == -1
+    assert f(*args, ctypes.byref(svg.svg_launch_opts(svg.SVG_ORDER_WORK, (1 << 20) + 4, 148)), None) == -1
