@@ -91,14 +91,17 @@ __device__ __forceinline__ float warp_sum(float x) {
 // Tensor-core form. Sampled rows x keys is a contraction (S = Q_rows K^T, then three P V), so one
 // CTA takes up to 128 sampled rows of one head (M = 128; rows past the list are padding) and one
 // chunk of the keys, streamed in 64-key tiles by TMA:
-//   warps 0-3  one thread per row: load the row's Q into shared memory (128-byte swizzle), then per
-//              tile load S from TMEM, and for each mask (dense, spatial, temporal) update that
-//              mask's running maximum and sum, compute P = 2^(S sl2 - m) on its kept keys in fp32
-//              and store it into that mask's two P buffers in shared memory as a bf16 pair,
-//              P = P_hi + P_lo with P_hi = bf16(P), P_lo = bf16(P - P_hi) (about 16 significant
-//              bits, so that the route's error sums keep the fp32 path's accuracy);
-//   warp 4     TMA producer of the K / V ring;
-//   warp 5     MMA issuer: S(e) = Q K(e)^T into TMEM (N = 64), then O_a += P_hi,a V(e) + P_lo,a V(e)
+//   warps 0-7  two threads per row (warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31; warp w
+//              takes columns [0, 32) of each tile, warp w + 4 columns [32, 64)): load the row's Q
+//              into shared memory (128-byte swizzle), then per tile load their half of S from TMEM,
+//              and for each mask (dense, spatial, temporal) trade the half-row maxima through
+//              shared memory, update that mask's running maximum and sum, compute P = 2^(S sl2 - m)
+//              on its kept keys in fp32 and store it into that mask's two P buffers in shared
+//              memory as a bf16 pair, P = P_hi + P_lo with P_hi = bf16(P), P_lo = bf16(P - P_hi)
+//              (about 16 significant bits, so that the route's error sums keep the fp32 path's
+//              accuracy);
+//   warp 8     TMA producer of the K / V ring;
+//   warp 9     MMA issuer: S(e) = Q K(e)^T into TMEM (N = 64), then O_a += P_hi,a V(e) + P_lo,a V(e)
 //              for the three masks into three TMEM accumulators. S(e + 1) is issued as soon as the softmax has
 //              loaded S(e) (P lives in shared memory), so it overlaps the softmax of tile e.
 // Every wait is bounded; the chunk state written out is the CUDA-core form's, so the same merge
@@ -106,9 +109,10 @@ __device__ __forceinline__ float warp_sum(float x) {
 constexpr int kRtRows = 128;
 constexpr int kRtKeys = kRouteKeys;
 constexpr int kRtStages = 4;
-constexpr int kRtThreads = 192;
-constexpr int kRtProducer = 4;
-constexpr int kRtMma = 5;
+constexpr int kRtThreads = 320;
+constexpr int kRtSoftmax = 256;  // two threads per row
+constexpr int kRtProducer = 8;
+constexpr int kRtMma = 9;
 
 template <int D>
 struct RtCfg {
@@ -117,7 +121,9 @@ struct RtCfg {
   static constexpr int kPBytes = kRtRows * kRtKeys * 2;    // one P buffer: 128 rows x 128 bytes
   static constexpr int kTileBytes = kRtKeys * D * 2;       // one K or V tile
   static constexpr int kDataBytes = kQBytes + 6 * kPBytes + kRtStages * kTileBytes;  // P_hi, P_lo per mask
-  static constexpr int kSmemBytes = kDataBytes + 256 /*barriers*/ + 1024 /*alignment*/;
+  static constexpr int kCtlBytes = 512;                    // barriers, abort flag, TMEM base
+  static constexpr int kXchBytes = 2 * 3 * 2 * kRtRows * 4;  // half-row maxima, final half-row sums
+  static constexpr int kSmemBytes = kDataBytes + kCtlBytes + kXchBytes + 1024 /*alignment*/;
   static constexpr uint32_t kSCol = 0;                     // S: 64 columns
   __host__ __device__ static constexpr uint32_t o_col(int a) { return 128u + (uint32_t)D * a; }
   static_assert(128 + 3 * D <= 512, "TMEM columns");
@@ -138,7 +144,8 @@ struct RouteTcParams {
 
 // barriers (8 bytes each): kv_full[NS], kv_empty[NS], q_full, s_full, s_free, p_ready[3], pv_done[3],
 // drain -- one p_ready / pv_done per mask, so that each mask's P store waits only for that mask's
-// previous P V
+// previous P V -- then xch[4][3]: the two threads of the rows of lane quarter q traded their half-row
+// maxima of mask a (64 arrivals per tile), and fin: every softmax thread wrote its half-row sums
 struct RtBar {
   uint32_t base;
   __device__ uint32_t kv_full(uint32_t i) const { return base + 8u * i; }
@@ -149,9 +156,12 @@ struct RtBar {
   __device__ uint32_t p_ready(int a) const { return base + 8u * (2 * kRtStages + 3 + a); }
   __device__ uint32_t pv_done(int a) const { return base + 8u * (2 * kRtStages + 6 + a); }
   __device__ uint32_t drain() const { return base + 8u * (2 * kRtStages + 9); }
-  static constexpr int kCount = 2 * kRtStages + 10;
+  __device__ uint32_t xch(int q, int a) const { return base + 8u * (2 * kRtStages + 10 + 3 * q + a); }
+  __device__ uint32_t fin() const { return base + 8u * (2 * kRtStages + 22); }
+  static constexpr int kCount = 2 * kRtStages + 23;
   static constexpr uint32_t kAbortOff = 8u * kCount;       // abort flag
   static constexpr uint32_t kTmemOff = kAbortOff + 8;      // TMEM base
+  static_assert(kTmemOff + 8 <= 512, "control block");
 };
 
 // Bits [lo - j0, hi - j0) of a 64-key tile starting at key j0 (clamped to the tile).
@@ -160,17 +170,6 @@ __device__ __forceinline__ uint64_t rt_range_bits(int j0, int lo, int hi) {
   if (b <= a) return 0ull;
   const uint64_t upto_b = b >= 64 ? ~0ull : ((1ull << b) - 1ull);
   return upto_b & ~((1ull << a) - 1ull);
-}
-
-// Keeps the kept keys' scores of one mask (bit j of keep) and folds them into the running state:
-// returns whether this thread's maximum grew past the rescale threshold (or had none yet).
-__device__ __forceinline__ bool rt_mask_max(const float* x, uint64_t keep, float m, float& m_new) {
-  float mx = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < kRtKeys; ++j)
-    if ((keep >> j) & 1ull) mx = fmaxf(mx, x[j]);
-  m_new = fmaxf(m, mx);
-  return (m_new > m) && (m == -INFINITY || m_new - m > kRescaleLog2);
 }
 
 template <int D>
@@ -182,6 +181,7 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
   const uint32_t sQ = sbase, sP = sQ + C::kQBytes, sRing = sP + 6 * C::kPBytes;
   RtBar b;
   b.base = sRing + kRtStages * C::kTileBytes;
+  const uint32_t sX = b.base + C::kCtlBytes;  // float [3][2][128] half-row maxima, then [3][2][128] sums
   uint8_t* ctl = smem_raw + (b.base - raw);
   const uint32_t abort_addr = b.base + RtBar::kAbortOff;
   int* status = P.status;
@@ -196,14 +196,16 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
       mbar_init(bar + i, 1);
       mbar_init(bar + kRtStages + i, 1);
     }
-    mbar_init(bar + 2 * kRtStages + 0, kRtRows);  // q_full: every softmax thread wrote its Q row
-    mbar_init(bar + 2 * kRtStages + 1, 1);        // s_full
-    mbar_init(bar + 2 * kRtStages + 2, kRtRows);  // s_free
+    mbar_init(bar + 2 * kRtStages + 0, kRtSoftmax);  // q_full: every softmax thread wrote its part of Q
+    mbar_init(bar + 2 * kRtStages + 1, 1);           // s_full
+    mbar_init(bar + 2 * kRtStages + 2, kRtSoftmax);  // s_free
     for (int a = 0; a < 3; ++a) {
-      mbar_init(bar + 2 * kRtStages + 3 + a, kRtRows);  // p_ready[a]
-      mbar_init(bar + 2 * kRtStages + 6 + a, 1);        // pv_done[a]
+      mbar_init(bar + 2 * kRtStages + 3 + a, kRtSoftmax);  // p_ready[a]
+      mbar_init(bar + 2 * kRtStages + 6 + a, 1);           // pv_done[a]
     }
     mbar_init(bar + 2 * kRtStages + 9, 1);  // drain
+    for (int i = 0; i < 12; ++i) mbar_init(bar + 2 * kRtStages + 10 + i, 64);  // xch[q][a]
+    mbar_init(bar + 2 * kRtStages + 22, kRtSoftmax);                           // fin
     *reinterpret_cast<volatile int*>(ctl + RtBar::kAbortOff) = 0;
     fence_mbar_init();
   }
@@ -319,17 +321,21 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- rows: Q, softmaxes, state out
-    const int lr = threadIdx.x;  // row within the block = TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int qd = warp & 3, half = warp >> 2;  // TMEM lane quarter; column half of each tile
+    const int lr = qd * 32 + lane;              // row within the block = TMEM lane
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    constexpr int kHalfCols = kRtKeys / 2;      // 32 score columns per thread
+    constexpr int kOCols = D / 2;               // output columns per thread
     const int ridx = blockIdx.x * kRtRows + lr;
     int r = ridx < P.n_rows ? __ldg(P.rows + ridx) : -1;
     if (r < 0 || r >= P.N) r = 0;  // padding and rows outside the sequence: any valid row, unused
     const int S = P.gs.S;
     const int ti = r / S, si = r - ti * S;
-    {  // Q row into the 128-byte-swizzle K-major tile: chunk c, row lr, 16-byte unit u at u ^ (lr % 8)
+    {  // this thread's chunks of the Q row into the 128-byte-swizzle K-major tile: chunk c, row lr,
+       // 16-byte unit u at u ^ (lr % 8)
       const uint4* src = reinterpret_cast<const uint4*>(P.q + ((size_t)h * P.N + r) * D);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
+      for (int c = half; c < C::kChunks; c += 2)
 #pragma unroll
         for (uint32_t u = 0; u < 8; ++u) {
           const uint4 v = __ldg(src + c * 8 + u);
@@ -339,6 +345,8 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
       fence_proxy_async_shared();
       mbar_arrive(b.q_full());
     }
+    float* xmax = reinterpret_cast<float*>(smem_raw + (sX - raw));  // [3][2][128]
+    float* xsum = xmax + 3 * 2 * kRtRows;                      // [3][2][128]
     float m[3] = {-INFINITY, -INFINITY, -INFINITY}, l[3] = {0.f, 0.f, 0.f};
     bool ok = true;
     for (int e = 0; e < ntiles; ++e) {
@@ -347,49 +355,60 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
         break;
       }
       tc_fence_after();
-      uint32_t sr[kRtKeys];
-      tmem_ld32(tmem + lane_off + C::kSCol, sr);
-      tmem_ld32(tmem + lane_off + C::kSCol + 32, sr + 32);
+      uint32_t sr[kHalfCols];
+      tmem_ld32(tmem + lane_off + C::kSCol + kHalfCols * half, sr);
       tmem_ld_wait();
       tmem_ld_fence32(sr);
-      tmem_ld_fence32(sr + 32);
       tc_fence_before();
       mbar_arrive(b.s_free());
-      float x[kRtKeys];
+      float x[kHalfCols];
 #pragma unroll
-      for (int j = 0; j < kRtKeys; ++j) x[j] = __uint_as_float(sr[j]) * P.sl2;
+      for (int j = 0; j < kHalfCols; ++j) x[j] = __uint_as_float(sr[j]) * P.sl2;
       // kept keys of each mask in this tile, as bit sets from their ranges of original key index
       // (key j = t * S + s): dense [j0, j_end); sink [0, F0 * S); spatial frames [ti - k, ti + k];
-      // temporal, in every frame t the tile touches, patches [si - b, si + b]
+      // temporal, in every frame t the tile touches, patches [si - b, si + b]; this thread's half
       const int j0 = j_begin + e * kRtKeys;
       const int jl = min(j0 + kRtKeys, j_end);  // end of this tile's keys
-      uint64_t keep[3];
-      keep[0] = rt_range_bits(j0, j0, jl);
-      const uint64_t sink = rt_range_bits(j0, 0, P.gs.F0 * S) & keep[0];
-      keep[1] = (rt_range_bits(j0, max(ti - P.gs.k, 0) * S, (min(ti + P.gs.k, P.gs.T - 1) + 1) * S) & keep[0]) | sink;
+      uint64_t keep64[3];
+      keep64[0] = rt_range_bits(j0, j0, jl);
+      const uint64_t sink = rt_range_bits(j0, 0, P.gs.F0 * S) & keep64[0];
+      keep64[1] = (rt_range_bits(j0, max(ti - P.gs.k, 0) * S, (min(ti + P.gs.k, P.gs.T - 1) + 1) * S) & keep64[0]) | sink;
       {
         const int s0 = max(si - P.gt.b, 0), s1 = min(si + P.gt.b, S - 1) + 1;
         uint64_t band = 0ull;
         for (int t = j0 / S; t * S < jl; ++t) band |= rt_range_bits(j0, t * S + s0, t * S + s1);
-        keep[2] = (band & keep[0]) | sink;
+        keep64[2] = (band & keep64[0]) | sink;
       }
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
-        float mn;
-        const bool need = rt_mask_max(x, keep[a], m[a], mn);
-        const bool rescale = __any_sync(0xffffffffu, need);
+        const uint32_t keep = (uint32_t)(keep64[a] >> (kHalfCols * half));
+        // the row's maximum: this half's, traded with the partner thread (bounded wait)
+        float hm = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kHalfCols; ++j)
+          if ((keep >> j) & 1u) hm = fmaxf(hm, x[j]);
+        xmax[(a * 2 + half) * kRtRows + lr] = hm;
+        mbar_arrive(b.xch(qd, a));
+        if (!__all_sync(0xffffffffu, wait_bar(b.xch(qd, a), (uint32_t)e & 1u, abort_addr, status))) {
+          ok = false;
+          break;
+        }
+        const float mx = fmaxf(hm, xmax[(a * 2 + (half ^ 1)) * kRtRows + lr]);
+        const float mn = fmaxf(m[a], mx);
+        const bool need = (mn > m[a]) && (m[a] == -INFINITY || mn - m[a] > kRescaleLog2);
+        const bool rescale = __any_sync(0xffffffffu, need);  // the same in both warps: same rows, same maxima
         float alpha = 1.f;
         if (rescale) {
           alpha = (mn == -INFINITY) ? 1.f : ex2f(m[a] - mn);
           l[a] *= alpha;
           m[a] = mn;
         }
-        uint32_t hi[kRtKeys / 2], lo[kRtKeys / 2];
+        uint32_t hi[kHalfCols / 2], lo[kHalfCols / 2];
         float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < kRtKeys; j += 2) {
-          const float p0 = ((keep[a] >> j) & 1ull) ? ex2f(x[j] - m[a]) : 0.f;
-          const float p1 = ((keep[a] >> (j + 1)) & 1ull) ? ex2f(x[j + 1] - m[a]) : 0.f;
+        for (int j = 0; j < kHalfCols; j += 2) {
+          const float p0 = ((keep >> j) & 1u) ? ex2f(x[j] - m[a]) : 0.f;
+          const float p1 = ((keep >> (j + 1)) & 1u) ? ex2f(x[j + 1] - m[a]) : 0.f;
           sum += p0 + p1;
           hi[j / 2] = pack_bf16(p0, p1);
           const float h0 = __uint_as_float(hi[j / 2] << 16), h1 = __uint_as_float(hi[j / 2] & 0xFFFF0000u);
@@ -402,32 +421,44 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        if (rescale) {
-          if (e > 0) {  // O_a holds the earlier tiles' P V (tile 0's MMA overwrites it)
-            const uint32_t tO = tmem + lane_off + C::o_col(a);
+        if (rescale && e > 0) {  // O_a holds the earlier tiles' P V (tile 0's MMA overwrites it); this
+                                 // thread rescales its half of the columns
+          const uint32_t tO = tmem + lane_off + C::o_col(a) + (uint32_t)(kOCols * half);
 #pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
-              uint32_t o[32];
-              tmem_ld32(tO + q * 32, o);
-              tmem_ld_wait();
-              tmem_ld_fence32(o);
+          for (int q = 0; q < kOCols / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
+            tmem_ld_wait();
+            tmem_ld_fence32(o);
 #pragma unroll
-              for (int y = 0; y < 32; ++y) o[y] = __float_as_uint(__uint_as_float(o[y]) * alpha);
-              tmem_st32(tO + q * 32, o);
-            }
-            tmem_st_wait();
+            for (int y = 0; y < 32; ++y) o[y] = __float_as_uint(__uint_as_float(o[y]) * alpha);
+            tmem_st32(tO + q * 32, o);
           }
+          tmem_st_wait();
         }
-        store_p_sw128<kRtKeys>(sP + (2 * a) * C::kPBytes, lr, hi);
-        store_p_sw128<kRtKeys>(sP + (2 * a + 1) * C::kPBytes, lr, lo);
+        // this thread's 64 bytes of the row (16-byte units 4 half .. 4 half + 3) in both buffers
+        const uint32_t rowb = (uint32_t)lr * 128u, sw = (uint32_t)lr & 7u;
+#pragma unroll
+        for (uint32_t u = 0; u < 4; ++u) {
+          const uint32_t off = rowb + (((4u * (uint32_t)half + u) ^ sw) << 4);
+          st_shared_v4(sP + (2 * a) * C::kPBytes + off, hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
+          st_shared_v4(sP + (2 * a + 1) * C::kPBytes + off, lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
+        }
         fence_proxy_async_shared();
         tc_fence_before();
         mbar_arrive(b.p_ready(a));
       }
       if (!ok) break;
     }
-    // ---- this chunk's state of the row: O (unnormalised), running max (log2 units), sum
+    // ---- this chunk's state of the row: O (unnormalised; each thread its half of the columns),
+    // running max (log2 units), sum (both threads' halves)
     bool done = ok && ntiles > 0;
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      if (done) xsum[(a * 2 + half) * kRtRows + lr] = l[a];
+    }
+    if (done) mbar_arrive(b.fin());
+    done = done && __all_sync(0xffffffffu, wait_bar(b.fin(), 0, abort_addr, status));
 #pragma unroll
     for (int a = 0; a < 3; ++a)
       done = done && __all_sync(0xffffffffu, wait_bar(b.pv_done(a), (uint32_t)(ntiles - 1) & 1u, abort_addr, status));
@@ -438,22 +469,22 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
 #pragma unroll 1
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q < kOCols / 32; ++q) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + C::o_col(a) + q * 32, o);
+          tmem_ld32(tmem + lane_off + C::o_col(a) + (uint32_t)(kOCols * half) + q * 32, o);
           tmem_ld_wait();
           tmem_ld_fence32(o);
           if (write) {  // (a row's state is 4-byte aligned only: scalar stores)
 #pragma unroll
-            for (int y = 0; y < 32; ++y) dst[a * (D + 2) + q * 32 + y] = __uint_as_float(o[y]);
+            for (int y = 0; y < 32; ++y) dst[a * (D + 2) + kOCols * half + q * 32 + y] = __uint_as_float(o[y]);
           }
         }
-        if (write) {
+        if (write && half == 0) {
           dst[a * (D + 2) + D] = m[a];
-          dst[a * (D + 2) + D + 1] = l[a];
+          dst[a * (D + 2) + D + 1] = xsum[(a * 2) * kRtRows + lr] + xsum[(a * 2 + 1) * kRtRows + lr];
         }
       }
-    } else if (ntiles == 0 && ridx < P.n_rows) {  // an empty chunk: nothing kept
+    } else if (ntiles == 0 && ridx < P.n_rows && half == 0) {  // an empty chunk: nothing kept
       float* dst = P.part + (((size_t)h * P.n_rows + ridx) * P.G + g) * 3 * (D + 2);
       for (int a = 0; a < 3; ++a) {
         for (int y = 0; y < D; ++y) dst[a * (D + 2) + y] = 0.f;

@@ -27,3 +27,18 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With SVG_CHECKED=1 the suite runs on the checked build (device-side bounds checks): every check
+    that failed anywhere in the session fails the run."""
+    if os.environ.get("SVG_CHECKED") != "1" or not _has_gpu():
+        return
+    import sys as _sys
+    mod = _sys.modules.get("block_sparse_spatio_flash_b200.svg")
+    if mod is None:
+        return
+    n = mod.svg_checks_failed(reset=False)
+    if n:
+        print(f"\nchecked build: {n} device-side bounds checks failed during the session")
+        session.exitstatus = 1
