@@ -9,7 +9,8 @@
 //
 // How (B200-specific, not the TPU design):
 //  * one CTA per SM, 320 threads, persistent; work items are (head, 256 query rows) taken
-//    from a global atomic counter in head-major order, each head's items heaviest first;
+//    from a global atomic counter in head-major order, each head's items heaviest first (or,
+//    as an option, longest processing time first over all heads);
 //  * warp 8 issues TMA loads (128-byte swizzle) of Q once per item and of K / V tiles into a
 //    shared-memory ring; warp 9 issues tcgen05 MMAs: S = Q K^T into TMEM, then O += P V with
 //    P read straight from TMEM;
@@ -22,6 +23,9 @@
 //    the result exact while making the correction rare;
 //  * every wait is bounded by a wall-clock limit; a timeout sets the status word and all
 //    roles drain their in-flight copies / MMAs and return.
+//  * fused token order: temporal heads read their tiles where the rows lie in the original order
+//    (whole runs of one patch's frames as 4-D boxes, edge rows gathered) and write O rows back to
+//    their original index.
 #include <cuda_bf16.h>
 #include <string.h>
 

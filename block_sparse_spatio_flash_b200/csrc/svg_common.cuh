@@ -23,7 +23,7 @@ namespace svg {
 constexpr uint32_t kTmMagic = 0x53564731u;  // "SVG1"
 constexpr int kMaxHeads = 4096;
 constexpr int64_t kMaxTokens = 1 << 22;
-constexpr int kPairRows = 256;  // query rows per item of the one-SM kernel: two 128-row halves
+constexpr int kPairRows = 256;  // query rows per item of the attention kernel: two 128-row halves
 constexpr int kHalfRows = 128;
 
 // Checked build (-DSVG_CHECKED=1, the library libsvgattn_checked.so): device-side bounds checks on
