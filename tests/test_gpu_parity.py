@@ -547,6 +547,53 @@ def test_work_order_gives_the_same_bytes_and_a_complete_trace(S, w, variant):
         gp.compare_rows(w.replace(sample_rows=128), q0, k0, v0, out.cpu(), None)
 
 
+def test_ablation_ordering_naive_slower_than_split_and_rounded_without_boundary(S):
+    """The pages' ablation ordering on spatial_75600: masking every visited tile (naive) is slower than
+    the full / boundary split, and the tile-aligned (rounded) map has no boundary tile while the exact
+    map has some."""
+    w = syn.SPATIAL_75K
+    dev = torch.device("cuda")
+    g, m, t = gp.geom_mask_tile(w)
+    routes = list(w.routes)
+    q, k, v = (x.to(dev) for x in syn.make_qkv(w))
+    maps = gp.build_maps(w, g, m, t, routes)
+    o = torch.empty_like(q)
+    sc = S.alloc_scratch()
+
+    def ms(mode):
+        for _ in range(2):
+            S.svg_attention_fwd(q, k, v, o, routes, maps[0], maps[1], g, m, t, mode=mode, scratch=sc)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record()
+        for _ in range(3):
+            S.svg_attention_fwd(q, k, v, o, routes, maps[0], maps[1], g, m, t, mode=mode, scratch=sc)
+        b_.record()
+        torch.cuda.synchronize()
+        return a_.elapsed_time(b_) / 3
+
+    split, naive = ms(S.SVG_MODE_SPLIT), ms(S.SVG_MODE_NAIVE)
+    assert S.svg_read_status(sc) == 0
+    assert naive > 1.2 * split, (naive, split)
+    exact = S.svg_tilemap_summary(maps[0])
+    gr, mr, tr = gp.geom_mask_tile(w, variant=syn.MASK_ROUNDED)
+    rounded = S.svg_tilemap_summary(gp.build_maps(w, gr, mr, tr, routes)[0])
+    assert rounded.n_boundary == 0 < exact.n_boundary
+
+
+def test_fused_order_1440p_equals_permuted_path_and_oracle(S):
+    """302,400 tokens (21 frames, 20-frame runs as boxes), 5 spatial + 5 temporal heads: the fused order
+    gives the permuted path's bytes, and the oracle's values on 256 seeded rows per head."""
+    w = syn.P1440
+    q, k, v = syn.make_qkv(w, seed_offset=91)
+    want, _, st = gp.run_path(w, q, k, v, lse=False)
+    assert st == 0
+    got, _, st = gp.run_fused(w, q, k, v, lse=False)
+    assert st == 0
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    del want
+    gp.compare_rows(w.replace(sample_rows=256), q, k, v, got, None)
+
+
 # ----------------------------------------------------------------------------- limits
 def test_max_heads_small_geometry(S):
     """4,096 heads (the ABI's limit) of a one-frame 8 x 8 geometry, alternating routes: the route bit
