@@ -270,6 +270,7 @@ struct FusedPlan {
   int kind;        // 0: inside the sink prefix, 1: gather every group, 2: runs and edge groups
   int n_box, u_a;  // whole runs u_a .. u_a + n_box - 1 (patch index = run index)
   uint32_t gmask;  // 4-row groups to gather (bit = group = lane)
+  int rr[4];       // this lane's gathered rows (original indices in the [heads * N, d] view)
 };
 
 template <int ROWS>
@@ -280,6 +281,7 @@ __device__ __forceinline__ FusedPlan fused_plan(const AttnParams& P, int p0, int
   f.n_box = 0;
   f.u_a = 0;
   f.gmask = 0;
+  f.rr[0] = f.rr[1] = f.rr[2] = f.rr[3] = 0;
   constexpr uint32_t kAll = ROWS / 4 >= 32 ? 0xFFFFFFFFu : ((1u << (ROWS / 4)) - 1u);
   if (p0 + ROWS <= pre) {
     f.kind = 0;
@@ -302,6 +304,22 @@ __device__ __forceinline__ FusedPlan fused_plan(const AttnParams& P, int p0, int
   const int r0 = 4 * lane;
   const bool need = r0 < ROWS && !(r0 >= c0 && r0 + 4 <= c1);
   f.gmask = __ballot_sync(0xFFFFFFFFu, need) & kAll;
+  return f;
+}
+
+// The plan and this lane's gathered rows for head `head`, tile rows [p0, p0 + ROWS).
+template <int ROWS>
+__device__ __forceinline__ FusedPlan fused_plan_rows(const AttnParams& P, int head, int p0, int lane) {
+  FusedPlan f = fused_plan<ROWS>(P, p0, lane);
+  if ((f.gmask >> lane) & 1u) {
+    const MaskGeom& g = P.g[SVG_ROUTE_TEMPORAL];
+    const int hrow = head * P.N;  // first row of the head in the [heads * N, d] view (fits: checked on the host)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f.rr[i] = hrow + orig_index(g, min(p0 + 4 * lane + i, P.N - 1));
+      if (!check_ok(f.rr[i] >= hrow && f.rr[i] < hrow + P.N, P.checks)) f.rr[i] = hrow;
+    }
+  }
   return f;
 }
 
@@ -330,15 +348,9 @@ __device__ __forceinline__ void fused_issue(const AttnParams& P, const FusedPlan
       tma_load_4d(dst + ch * (ROWS * 128) + row * 128u, box_map, bar, ch * 64, u, P.run_t0, head);
   }
   if ((f.gmask >> lane) & 1u) {
-    const int hrow = head * P.N;  // first row of the head in the [heads * N, d] view (fits: checked on the host)
-    int rr[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      rr[i] = hrow + orig_index(g, min(p0 + 4 * lane + i, P.N - 1));
-      if (!check_ok(rr[i] >= hrow && rr[i] < hrow + P.N, P.checks)) rr[i] = hrow;
-    }
     for (int ch = 0; ch < CHUNKS; ++ch)
-      tma_gather4(dst + ch * (ROWS * 128) + (uint32_t)lane * 512u, row_map, bar, ch * 64, rr[0], rr[1], rr[2], rr[3]);
+      tma_gather4(dst + ch * (ROWS * 128) + (uint32_t)lane * 512u, row_map, bar, ch * 64, f.rr[0], f.rr[1], f.rr[2],
+                  f.rr[3]);
   }
 }
 
@@ -467,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         for (int h = 0; h < 2; ++h) {
           if ((h == 0 ? inf.nA : inf.nB) == 0) continue;
           if (gat) {
-            qpl[h] = fused_plan<kHalfRows>(P, inf.pair * kPairRows + h * kHalfRows, lane);
+            qpl[h] = fused_plan_rows<kHalfRows>(P, inf.head, inf.pair * kPairRows + h * kHalfRows, lane);
             qbytes += fused_bytes<kHalfRows, C::kChunks>(P, qpl[h]);
           } else {
             qbytes += (uint32_t)C::kQHalfBytes;
@@ -492,12 +504,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       // K / V loads in the order the MMA warp consumes them: K(e), V(e) per entry; with P in
       // shared memory S(e+1) comes before P V(e): K(0), then K(e+1), V(e) per entry.
-      // the last two entries' key-tile rows, {entry, row0} by entry parity: each entry's is
-      // worked out once
+      // the last two entries' key-tile rows, {entry, row0} by entry parity, and in fused order their
+      // copy plans: each entry's are worked out once, for its K and its V tile
       int ca[2] = {-1, 0}, cb[2] = {-1, 0};
-      auto fill = [&](int (&cc)[2], int e) {
+      FusedPlan pa, pb;
+      auto fill = [&](int (&cc)[2], FusedPlan& pl, int e) {
         cc[0] = e;
         cc[1] = (int)ent_kt(get_entry<BK>(P, inf, e)) * BK;
+        if (gat) pl = fused_plan_rows<BK>(P, inf.head, cc[1], lane);
       };
       bool ok = true;
       for (int n = 0; n < 2 * inf.count && ok; ++n) {
@@ -517,12 +531,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           w = m & 1;
         }
         int row0;
+        FusedPlan kpl;
         if ((e & 1) == 0) {
-          if (ca[0] != e) fill(ca, e);
+          if (ca[0] != e) fill(ca, pa, e);
           row0 = ca[1];
+          kpl = pa;
         } else {
-          if (cb[0] != e) fill(cb, e);
+          if (cb[0] != e) fill(cb, pb, e);
           row0 = cb[1];
+          kpl = pb;
         }
         const uint32_t st = kv_pos % NS, phs = (kv_pos / NS) & 1u;
         if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.kv_empty(st), phs ^ 1u, abort_addr, status) : 0,
@@ -530,8 +547,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           ok = false;
           break;
         }
-        FusedPlan kpl;
-        if (gat) kpl = fused_plan<BK>(P, row0, lane);
         if (lane == 0)
           mbar_expect_tx(c.kv_full(st), gat ? fused_bytes<BK, C::kChunks>(P, kpl) : (w == 0 ? C::kKBytes : C::kVBytes));
         __syncwarp();
