@@ -314,6 +314,8 @@ int run_attention(const void* q, const void* k, const void* v, void* o, float* l
     // in the fully space-major order; runs shorter than 4 rows are gathered instead
     const bool fsm = mask->layout == SVG_LAYOUT_FULL_SPACE_MAJOR;
     const int run = fsm ? geom->frames : geom->frames - mask->sink_frames;
+    P.run_div = make_fastdiv(run > 0 ? (uint32_t)run : 1u);
+    P.runs = run > 0 ? (N - (fsm ? 0 : mask->sink_frames * geom->grid_h * geom->grid_w)) / run : 0;
     if (run >= 4 && run <= 256) {
       const int S = geom->grid_h * geom->grid_w;
       P.run_len = run;

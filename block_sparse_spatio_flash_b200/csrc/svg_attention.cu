@@ -294,10 +294,9 @@ __device__ __forceinline__ FusedPlan fused_plan(const AttnParams& P, int p0, int
   }
   f.kind = 2;
   const int q0 = p0 - pre;
-  const int u_a = (q0 + R - 1) / R;  // first run that starts inside the tile
-  int u_end = (q0 + ROWS) / R;       // runs [u_a, u_end) end inside the tile
-  const int runs = (g.N - pre) / R;
-  if (u_end > runs) u_end = runs;
+  const int u_a = (int)fastdiv((uint32_t)(q0 + R - 1), P.run_div);  // first run that starts inside the tile
+  int u_end = (int)fastdiv((uint32_t)(q0 + ROWS), P.run_div);       // runs [u_a, u_end) end inside the tile
+  if (u_end > P.runs) u_end = P.runs;
   f.u_a = u_a;
   f.n_box = u_end > u_a ? u_end - u_a : 0;
   const int c0 = f.n_box ? u_a * R - q0 : 0, c1 = f.n_box ? u_end * R - q0 : 0;  // rows the boxes cover
@@ -305,6 +304,20 @@ __device__ __forceinline__ FusedPlan fused_plan(const AttnParams& P, int p0, int
   const bool need = r0 < ROWS && !(r0 >= c0 && r0 + 4 <= c1);
   f.gmask = __ballot_sync(0xFFFFFFFFu, need) & kAll;
   return f;
+}
+
+// Original index of the token at position p of a temporal head's order (orig_index with the run
+// division done by fastdiv).
+__device__ __forceinline__ int temporal_orig_index(const AttnParams& P, const MaskGeom& g, int p) {
+  if (g.layout == SVG_LAYOUT_FULL_SPACE_MAJOR) {
+    const int s = (int)fastdiv((uint32_t)p, P.run_div);
+    return (p - s * g.T) * g.S + s;
+  }
+  const int pre = g.F0 * g.S;
+  if (p < pre) return p;
+  const int q = p - pre;
+  const int s = (int)fastdiv((uint32_t)q, P.run_div);
+  return (g.F0 + q - s * (g.T - g.F0)) * g.S + s;
 }
 
 // The plan and this lane's gathered rows for head `head`, tile rows [p0, p0 + ROWS).
@@ -316,7 +329,7 @@ __device__ __forceinline__ FusedPlan fused_plan_rows(const AttnParams& P, int he
     const int hrow = head * P.N;  // first row of the head in the [heads * N, d] view (fits: checked on the host)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      f.rr[i] = hrow + orig_index(g, min(p0 + 4 * lane + i, P.N - 1));
+      f.rr[i] = hrow + temporal_orig_index(P, g, min(p0 + 4 * lane + i, P.N - 1));
       if (!check_ok(f.rr[i] >= hrow && f.rr[i] < hrow + P.N, P.checks)) f.rr[i] = hrow;
     }
   }

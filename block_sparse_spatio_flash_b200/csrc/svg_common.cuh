@@ -167,6 +167,33 @@ struct TmLayout {
   int nq, nk, npairs;
 };
 
+// Division of 32-bit unsigned numbers by a divisor d >= 1 fixed per launch, by one multiply-high,
+// an add and two shifts (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", 1994, the round-up method for N = 32): with l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1, t = hi32(m n), the quotient is (t + ((n - t) >> min(l, 1)))
+// >> max(l - 1, 0), exact for every 32-bit n.
+struct FastDiv {
+  uint32_t m, s1, s2, d;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (1ull << l) < d) ++l;
+  FastDiv f;
+  f.m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d) + 1);
+  f.s1 = l < 1 ? l : 1;
+  f.s2 = l > 0 ? l - 1 : 0;
+  f.d = d;
+  return f;
+}
+__host__ __device__ inline uint32_t fastdiv(uint32_t n, const FastDiv& f) {
+#if defined(__CUDA_ARCH__)
+  const uint32_t t = __umulhi(n, f.m);
+#else
+  const uint32_t t = (uint32_t)(((uint64_t)n * f.m) >> 32);
+#endif
+  return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
 // Records a failed CUDA call (what + error) for svg_last_cuda_error; returns SVG_ERR_CUDA.
 int record_cuda_error(const char* what, int cuda_error);
 
@@ -218,6 +245,10 @@ struct AttnParams {
   // apart in the original order) in one tiled copy; run_len = 0 when runs are not copied as boxes
   CUtensorMap tm_q4, tm_k4, tm_v4;
   int run_len, run_t0;
+  // fused order: division by the length of a patch's run of frames (T in the fully space-major
+  // order, T - F0 after the sink prefix; d = 1 when there is none), and the number of runs
+  FastDiv run_div;
+  int runs;
   int fused;
   // QK^T operands in e4m3 (one byte per element): tm_q / tm_k then describe 1-byte tensors
   int qk8;
