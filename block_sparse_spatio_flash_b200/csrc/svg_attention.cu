@@ -8,12 +8,12 @@
 // memory O(N d).
 //
 // How (B200-specific, not the TPU design):
-//  * one CTA per SM, 320 threads, persistent; work items are (head, 256 query rows) taken
+//  * one CTA per SM, 352 threads, persistent; work items are (head, 256 query rows) taken
 //    from a global atomic counter in head-major order, each head's items heaviest first (or,
 //    as an option, longest processing time first over all heads);
-//  * warp 8 issues TMA loads (128-byte swizzle) of Q once per item and of K / V tiles into a
-//    shared-memory ring; warp 9 issues tcgen05 MMAs: S = Q K^T into TMEM, then O += P V with
-//    P read straight from TMEM;
+//  * warp 8 issues TMA loads (128-byte swizzle) of Q once per item and of the K tiles, warp 10
+//    those of the V tiles, into a shared-memory ring; warp 9 issues tcgen05 MMAs: S = Q K^T
+//    into TMEM, then O += P V with P read straight from TMEM;
 //  * warps 0-3 and 4-7 are two softmax groups, one per 128-row half, one thread per query
 //    row (= TMEM lane). While one group turns its S into P, the tensor core computes the
 //    other half's S and P V, so MMA and exponentials overlap;
@@ -33,9 +33,10 @@
 
 namespace svg {
 
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
+constexpr int kThreads = 352;
+constexpr int kProducerWarp = 8;   // claims the items, loads Q and the K tiles
 constexpr int kMmaWarp = 9;
+constexpr int kProducer2Warp = 10;  // loads the V tiles of the items warp 8 publishes
 
 
 // QK8: Q and K in e4m3 (one byte per element, d = 128: one 128-byte swizzle chunk per row), QK^T on
@@ -82,7 +83,7 @@ struct ItemInfo {
 //   2NS + 6 + h    o_done[h]     last P V of half h complete (PS: every P V of half h, pv_done)
 //   2NS + 8 + h    o_free[h]     epilogue finished reading O_h (128 arrivals)
 //   2NS + 10 + i   item_full[i]  work item published in slot i
-//   2NS + 12 + i   item_empty[i] slot i read by the MMA warp and the 8 softmax warps
+//   2NS + 12 + i   item_empty[i] slot i read by the MMA warp, the 8 softmax warps and the V producer
 //   2NS + 14       drain         final MMA completion
 //   2NS + 15       never         completed by nothing (test hook: a wait that runs out)
 //   2NS + 16 + h   s_free[h]     (PS) S_h loaded by the softmax, its TMEM columns free (128 arrivals)
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       mbar_init(b + 6 + h, 1);     // o_done
       mbar_init(b + 8 + h, 128);   // o_free
       mbar_init(b + 10 + h, 1);    // item_full
-      mbar_init(b + 12 + h, 9);    // item_empty
+      mbar_init(b + 12 + h, 10);   // item_empty
     }
     mbar_init(b + 14, 1);  // drain
     mbar_init(b + 15, 1);  // never
@@ -442,21 +443,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const uint32_t tmem = *reinterpret_cast<uint32_t*>(ctl_gen + K::kTmemOff);
   const bool skip_all = *reinterpret_cast<int*>(ctl_gen + K::kBadWsOff) != 0;
 
-  if (!skip_all && warp == kProducerWarp) {
+  if (!skip_all && (warp == kProducerWarp || warp == kProducer2Warp)) {
     // ------------------------------------------------------------------ producer
     // Lane 0 takes the waits, the work counter and the transaction counts; the results are
     // broadcast so that the whole warp follows the same control flow. Tiled loads are issued by
     // lane 0; in fused token order a temporal item's tiles are read where their rows lie
     // (fused_plan / fused_issue: whole runs as boxes by lanes 0.., edge groups gathered by lane L
     // for rows 4L .. 4L + 3).
+    // Two producer warps share the ring: warp 8 claims and publishes the items, loads Q and every K
+    // tile; warp 10 reads the published items and loads every V tile. Both count the ring positions
+    // of every tile, so each tile keeps the position (slot and phase) the MMA warp reads it at.
+    const bool vw = warp == kProducer2Warp;
+    const int my_w = vw ? 1 : 0;
     uint32_t kv_pos = 0, q_iter = 0, tr_items = 0, tr_tiles = 0;
+    uint32_t mine = 0;  // bit i: this warp filled ring position kv_pos - 1 - i
     bool q_issued = false;
     for (uint32_t it = 0;; ++it) {
       const uint32_t slot = it & 1u, ph = (it >> 1) & 1u;
+      ItemInfo inf;
+      if (vw) {  // the item warp 8 published in this slot
+        if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.item_full(slot), ph, abort_addr, status) : 0, 0))
+          break;
+        inf = items[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(c.item_empty(slot));
+        if (!inf.valid) break;
+      } else {
       if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.item_empty(slot), ph ^ 1u, abort_addr, status) : 0,
                        0))
         break;
-      ItemInfo inf;
       if (P.order == kOrderWork) {
         int wc = 0;
         uint32_t wpos = 0;
@@ -480,8 +495,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
       }
       if (!inf.valid) break;
+      }
       const bool gat = P.fused && inf.cls == SVG_ROUTE_TEMPORAL;
-      if (inf.nA + inf.nB > 0) {
+      if (!vw && inf.nA + inf.nB > 0) {
         if (!__shfl_sync(0xffffffffu, lane == 0 ? (int)wait_bar(c.q_free(), (q_iter & 1u) ^ 1u, abort_addr, status) : 0,
                          0))
           break;
@@ -543,6 +559,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           e = (m >> 1) + ((m & 1) ^ 1);
           w = m & 1;
         }
+        if (w != my_w) {  // the other producer's tile: its position only
+          ++kv_pos;
+          mine <<= 1;
+          continue;
+        }
         int row0;
         FusedPlan kpl;
         if ((e & 1) == 0) {
@@ -577,18 +598,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
         }
         ++kv_pos;
+        mine = (mine << 1) | 1u;
       }
       if (!ok) break;
     }
     if (lane == 0 && ld_shared_volatile(abort_addr)) {  // let issued copies land before the CTA may exit
+      // (each producer drains the positions it filled among the last NS)
       const uint32_t n = kv_pos < (uint32_t)NS ? kv_pos : (uint32_t)NS;
       for (uint32_t i = 0; i < n; ++i) {
+        if (!((mine >> i) & 1u)) continue;
         const uint32_t pos = kv_pos - 1 - i;
         drain_bar(c.kv_full(pos % NS), (pos / NS) & 1u);
       }
       if (q_issued) drain_bar(c.q_full(), (q_iter - 1) & 1u);
     }
-    if (lane == 0) {  // this CTA's share of the work, for the optional trace
+    if (lane == 0 && !vw) {  // this CTA's share of the work, for the optional trace
       *reinterpret_cast<uint32_t*>(ctl_gen + K::kTraceOff) = tr_items;
       *reinterpret_cast<uint32_t*>(ctl_gen + K::kTraceOff + 4) = tr_tiles;
     }
