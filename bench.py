@@ -405,7 +405,7 @@ def main():
 # spatial_75600 (128 x 128 tiles, split mode), scaled to the launch's heads: traffic grows with the
 # heads processed. Valid only for the kernel sources that were captured (their SHA-256 prefix);
 # after any change to them the field is null until the capture is repeated.
-CAPTURED_TRAFFIC = {"sources_sha256": "ace7218135b2ee6b", "bytes_per_head": 145.19168e6 / 2,
+CAPTURED_TRAFFIC = {"sources_sha256": "93f52114e7858f0a", "bytes_per_head": 138.852352e6 / 2,
                     "workload": "spatial_75600", "bq": 128, "bk": 128, "mode": "split"}
 
 
