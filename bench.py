@@ -136,6 +136,19 @@ def time_events(fn, iters, stream):
     return s.elapsed_time(e) / iters
 
 
+def time_interleaved(fns, iters, rounds, stream):
+    """Median over `rounds` of the mean ms per call over `iters` calls, for each callable of `fns`
+    (a dict), after one untimed call each; the callables take turns within every round, so that
+    clock and power changes during the measurement fall on all of them alike."""
+    for fn in fns.values():
+        fn()
+    times = {k: [] for k in fns}
+    for _ in range(rounds):
+        for k, fn in fns.items():
+            times[k].append(time_events(fn, iters, stream))
+    return {k: statistics.median(v) for k, v in times.items()}
+
+
 def workload_flops(w, summaries):
     """(effective, visited, executed) FLOP per call: 4*d*pairs; retained / in-range visited area /
     MMA work actually issued (128-row halves x bk key tiles)."""
@@ -604,12 +617,13 @@ def other_workloads(S, P, stream, dev):
             S.svg_build_tilemap(g, m, t, c, ws[c])
             summ[c] = S.svg_tilemap_summary(ws[c])
         sc = S.alloc_scratch(dev)
-        ms = time_events(lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, scratch=sc), 5,
-                         stream)
-        # the same call with the permutation inside the kernel (original-order tensors)
-        ms_fused = time_events(
-            lambda: S.svg_attention_fwd_fused(q, k, v, o, routes, ws[0], ws[1], g, m, t, scratch=sc), 3, stream)
-        ms_perm = time_events(lambda: S.svg_permute(q, qp, routes, g, m), 3, stream)
+        # the permuted layout's attention, the same call with the permutation inside the kernel
+        # (original-order tensors) and one permutation pass, taking turns
+        tm = time_interleaved({
+            "attn": lambda: S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, scratch=sc),
+            "fused": lambda: S.svg_attention_fwd_fused(q, k, v, o, routes, ws[0], ws[1], g, m, t, scratch=sc),
+            "perm": lambda: S.svg_permute(q, qp, routes, g, m)}, 2, 3, stream)
+        ms, ms_fused, ms_perm = tm["attn"], tm["fused"], tm["perm"]
         eff, vis, _ = workload_flops(w, summ)
         res[w.name] = {"ms": ms, "effective_tflops": eff / (ms * 1e-3) / 1e12,
                        "visited_tflops": vis / (ms * 1e-3) / 1e12,

@@ -581,13 +581,17 @@ int svg_route_heads(const void* q, const void* k, const void* v, int32_t heads, 
 
 // ---------------------------------------------------------------------------------------
 // Host-buffer entry point: chunks of heads flow through three library streams (copies in,
-// compute, copies out) and two device slots, so the copies of one chunk overlap the
-// permutation and attention of the neighbouring chunks.
+// compute, copies out) and three device slots, so the copies of one chunk overlap the
+// permutation and attention of the neighbouring chunks. With two slots the copy in of chunk
+// c + 2 had to wait for the copy out of chunk c, i.e. for its attention: the copy-in stream,
+// the bound of the whole call, stalled every chunk; a third slot lets it run ahead.
 namespace {
+
+constexpr int kHostSlots = 3;
 
 struct HostPipe {
   cudaStream_t in, comp, out;
-  cudaEvent_t h2d[2], done[2], d2h[2];
+  cudaEvent_t h2d[kHostSlots], done[kHostSlots], d2h[kHostSlots];
   std::mutex call;  // one host-buffer call per device at a time: the streams and events are shared
 };
 
@@ -605,7 +609,7 @@ HostPipe* host_pipe(int* rc) {
     cudaError_t e = cudaStreamCreateWithFlags(&hp->in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp->comp, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp->out, cudaStreamNonBlocking);
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+    for (int i = 0; i < kHostSlots && e == cudaSuccess; ++i) {
       e = cudaEventCreateWithFlags(&hp->h2d[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp->done[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp->d2h[i], cudaEventDisableTiming);
@@ -634,7 +638,7 @@ __global__ void keep_status(const int* launch_status, int* call_status) {
 size_t svg_attention_host_buffer_bytes(int64_t tokens, int32_t d, int32_t chunk_heads) {
   if (tokens < 1 || tokens > kMaxTokens || (d != 64 && d != 128) || chunk_heads < 1 || chunk_heads > kMaxHeads)
     return 0;
-  return 2 * 7 * chunk_tensor_bytes(tokens, d, chunk_heads) + kScratchBytes + 256;
+  return kHostSlots * 7 * chunk_tensor_bytes(tokens, d, chunk_heads) + kScratchBytes + 256;
 }
 
 int svg_attention_fwd_host(const void* h_q, const void* h_k, const void* h_v, void* h_o, int32_t heads,
@@ -661,8 +665,8 @@ int svg_attention_fwd_host(const void* h_q, const void* h_k, const void* h_v, vo
 
   const size_t ta = chunk_tensor_bytes(tokens, d, ch);
   uint8_t* buf = static_cast<uint8_t*>(d_buf);
-  void* scratch = buf + 2 * 7 * ta;
-  int* call_status = reinterpret_cast<int*>(buf + 2 * 7 * ta + kScratchBytes);
+  void* scratch = buf + kHostSlots * 7 * ta;
+  int* call_status = reinterpret_cast<int*>(buf + kHostSlots * 7 * ta + kScratchBytes);
   const size_t head_bytes = (size_t)tokens * d * 2;
   const int nchunks = (heads + ch - 1) / ch;
   cudaError_t e = cudaSuccess;
@@ -679,7 +683,7 @@ int svg_attention_fwd_host(const void* h_q, const void* h_k, const void* h_v, vo
   for (int c = 0; c < nchunks; ++c) {
     const int h0 = c * ch, hn = (heads - h0) < ch ? (heads - h0) : ch;
     const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hn * head_bytes;
-    const int s = c & 1;
+    const int s = c % kHostSlots;
     uint8_t* base = buf + (size_t)s * 7 * ta;
     uint8_t *qo = base, *ko = base + ta, *vo = base + 2 * ta;
     uint8_t *qp = base + 3 * ta, *kp = base + 4 * ta, *vp = base + 5 * ta, *op = base + 6 * ta;
@@ -687,7 +691,7 @@ int svg_attention_fwd_host(const void* h_q, const void* h_k, const void* h_v, vo
     bool perm = false;
     for (int h = 0; h < hn; ++h) perm |= routes[h] != 0;
     // copies in: the slot's previous chunk must have left the device (its copy out read qo or op)
-    if (c >= 2) SVG_HOST_TRY(cudaStreamWaitEvent(hp->in, hp->d2h[s], 0), "cudaStreamWaitEvent(in)");
+    if (c >= kHostSlots) SVG_HOST_TRY(cudaStreamWaitEvent(hp->in, hp->d2h[s], 0), "cudaStreamWaitEvent(in)");
     SVG_HOST_TRY(cudaMemcpyAsync(qo, static_cast<const uint8_t*>(h_q) + off, bytes, cudaMemcpyHostToDevice, hp->in),
                  "cudaMemcpyAsync(q in)");
     SVG_HOST_TRY(cudaMemcpyAsync(ko, static_cast<const uint8_t*>(h_k) + off, bytes, cudaMemcpyHostToDevice, hp->in),

@@ -290,7 +290,7 @@ int svg_route_heads(const void *q, const void *k, const void *v, int32_t heads, 
  * their token order, runs svg_attention_fwd, takes O back to the original order and copies it
  * to the host; the same computation as svg_permute + svg_attention_fwd + svg_permute(inverse)
  * on device buffers, with bitwise-identical results. Heads go through in chunks of
- * `chunk_heads`, on three streams owned by the library (copies in, compute, copies out) and two
+ * `chunk_heads`, on three streams owned by the library (copies in, compute, copies out) and three
  * device slots, so that one chunk's copies overlap the neighbouring chunks' compute
  * ("Sources & evidence" of the case study: the pages time the attention kernel alone and leave
  * out host transfers; this call is what a user without device buffers runs).
@@ -319,8 +319,9 @@ int svg_attention_fwd_host(const void *h_q, const void *h_k, const void *h_v, vo
  * all in the ORIGINAL frame-major order for every head, and no svg_permute pass is needed. The
  * pages' kernel runs temporal heads on permuted tokens and leaves the reordering out of its
  * timings ("routing, token permutation" excluded, "Sources & evidence"); here temporal heads
- * read each K/V/Q tile's rows where they lie (4-row TMA gathers at their original indices) and
- * write each O row back to its original index, so the arithmetic, tile by tile, is that of
+ * read each K/V/Q tile's rows where they lie (one patch's run of frames as one strided TMA box,
+ * 4-row TMA gathers for the partial runs at tile edges) and write each O row back to its
+ * original index, so the arithmetic, tile by tile, is that of
  * svg_permute + svg_attention_fwd + svg_permute(inverse) and the results are bitwise equal.
  * Arguments as svg_attention_fwd; lse (nullable) is [heads, tokens] in original order.
  * SVG_ERR_UNSUPPORTED when heads * tokens exceeds 2^31 - 1 (rows are gathered through a

@@ -152,7 +152,7 @@ def test_host_entry_argument_checks(svg):
     lib = ctypes.CDLL(svg.LIB_PATH)
     hb = svg.svg_attention_host_buffer_bytes
     one = (512 * 64 * 2 + 255) // 256 * 256
-    assert hb(512, 64, 1) == 2 * 7 * one + 256 + 256
+    assert hb(512, 64, 1) == 3 * 7 * one + 256 + 256
     assert hb(512, 96, 1) == 0 and hb(512, 64, 0) == 0 and hb(0, 64, 1) == 0
     f = lib.svg_attention_fwd_host
     f.argtypes = svg._sig["svg_attention_fwd_host"][1]

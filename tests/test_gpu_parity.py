@@ -442,7 +442,7 @@ def test_route_several_key_chunks(S, d):
 
 # ----------------------------------------------------------------------------- host-buffer entry
 @pytest.mark.parametrize("chunk", [1, 3, 4, 9])
-@pytest.mark.parametrize("routes", [(0, 1, 0, 1), (0, 0, 0, 0), (1, 1, 0, 1)])
+@pytest.mark.parametrize("routes", [(0, 1, 0, 1), (0, 0, 0, 0), (1, 1, 0, 1), (0, 1, 1, 0, 0, 1, 0)])
 def test_host_entry_matches_device_path(S, chunk, routes):
     """svg_attention_fwd_host (pinned host buffers, chunked pipeline) gives exactly the bytes of
     the device-buffer path, and so the oracle's values."""
