@@ -2,11 +2,13 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload spatial_75600|temporal_75600|mixed_75600|p1440_302400]
-                    [--bq 128 --bk 128] [--mode split|naive] [--no-extras]
+                    [--bq 128 --bk 128] [--mode split|naive] [--fused] [--no-extras]
 
 A step is one call of svg_attention_fwd (split mode: full tiles unmasked, boundary tiles
 masked) over the whole workload, Q/K/V/O resident in HBM (774 MB at 75,600 tokens, larger
-than the 126 MB L2, so no flush is needed between steps). Tile maps are built once per
+than the 126 MB L2, so no flush is needed between steps). With --fused a step is one call of
+svg_attention_fwd_fused on original-order tensors instead (temporal heads' token permutation
+inside the kernel). Tile maps are built once per
 geometry (the design caches them) and timed separately, as are the token permutation, the
 dense baseline, the naive and the rounded modes. Multi-GPU runs are independent replicas
 (the path has no exchange step): every rank runs the same workload; the step time is the
@@ -201,7 +203,8 @@ def workload_config(w, args):
     return {"workload": w.name, "tokens": w.tokens, "heads": w.heads, "d": w.d,
             "routes": "".join("S" if r == 0 else "T" for r in w.routes),
             "frame_window": w.frame_window, "spatial_band": w.spatial_band, "sink_frames": w.sink_frames,
-            "bq": w.bq, "bk": w.bk, "mode": args.mode}
+            "bq": w.bq, "bk": w.bk, "mode": args.mode,
+            **({"token_order": "fused"} if getattr(args, "fused", False) else {})}
 
 
 def run_reference(args, w, world, rank):
@@ -246,6 +249,8 @@ def main():
     ap.add_argument("--bq", type=int, default=128)
     ap.add_argument("--bk", type=int, default=128)
     ap.add_argument("--mode", default="split", choices=["split", "naive"])
+    ap.add_argument("--fused", action="store_true",
+                    help="time svg_attention_fwd_fused (token permutation inside the kernel) as the step")
     ap.add_argument("--chunk-heads", type=int, default=1, help="heads per chunk of the host-buffer pipeline")
     ap.add_argument("--no-extras", action="store_true", help="skip the side measurements")
     ap.add_argument("--quick", action="store_true",
@@ -318,10 +323,15 @@ def main():
     if plan is not None and world > 1:
         o_all = torch.empty((plan.heads,) + tuple(o.shape[1:]), dtype=o.dtype, device=dev)
 
+    o_orig = torch.empty_like(q) if args.fused else None
+
     def step():
-        S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, mode=mode, scratch=scratch)
+        if args.fused:
+            S.svg_attention_fwd_fused(q, k, v, o_orig, routes, ws[0], ws[1], g, m, t, mode=mode, scratch=scratch)
+        else:
+            S.svg_attention_fwd(qp, kp, vp, o, routes, ws[0], ws[1], g, m, t, mode=mode, scratch=scratch)
         if o_all is not None:  # every rank ends the step with all heads' O
-            shard.gather_heads(o, plan, out=o_all)
+            shard.gather_heads(o_orig if args.fused else o, plan, out=o_all)
 
     for _ in range(args.warmup):
         step()
@@ -355,7 +365,8 @@ def main():
     achieved = vis_flop / (statistics.mean(per_step) * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": captured_traffic(w, args),
-                "kernel": f"attn_kernel<128,128> ({args.mode}, {kernel_variant()} schedule)",
+                "kernel": f"attn_kernel<128,128> ({args.mode}{', fused token order' if args.fused else ''}, "
+                          f"{kernel_variant()} schedule)",
                 "flop_definition": "4*d*(in-range area of visited tiles)", "peak_kind": f"{peak_kind} bf16 burst"}
 
     if args.route_calls > 0:
@@ -440,7 +451,8 @@ def kernel_variant() -> str:
 def captured_traffic(w, args):
     c = CAPTURED_TRAFFIC
     if (kernel_sources_sha() != c["sources_sha256"] or w.name != c["workload"] or args.bq != c["bq"]
-            or args.bk != c["bk"] or args.mode != c["mode"] or kernel_variant() != "default"):
+            or args.bk != c["bk"] or args.mode != c["mode"] or kernel_variant() != "default"
+            or getattr(args, "fused", False)):
         return None
     return c["bytes_per_head"] * w.heads
 
