@@ -21,7 +21,8 @@
 namespace svg {
 
 constexpr int kRouteKeys = 64;      // keys per tile
-constexpr int kRouteMaxChunks = 32;
+constexpr int kRouteMaxChunks = 32;  // at most one chunk per lane of the merge kernel's warp
+static_assert(kRouteMaxChunks <= 32, "route_merge_kernel keeps one chunk per lane");
 constexpr int kRouteChunkKeys = 2048;
 
 // Key chunks per row block: enough blocks to fill the GPU at the pages' sizes, at most 32.
@@ -84,6 +85,16 @@ struct RouteParams {
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
   return x;
 }
 
@@ -499,42 +510,48 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const __grid_co
   if (warp == kRtMma) tmem_dealloc(tmem, 512);
 }
 
-// One warp per (sampled row, head): combine the chunks' states of each mask, then the row's
-// squared errors of the sparse outputs against the dense one.
-__global__ void route_merge_kernel(const RouteParams P) {
-  const int ridx = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
+// One block of three warps per (sampled row, head): warp a combines the chunks' states of mask a
+// (dense, spatial, temporal), then warp 0 takes the row's squared errors of the sparse outputs
+// against the dense one. Lane g holds chunk g's maximum and sum (at most 32 chunks), so the common
+// maximum and the rescaled sum are warp reductions; the chunks' partial outputs are read four
+// chunks at a time, their loads in flight together.
+__global__ void __launch_bounds__(96) route_merge_kernel(const RouteParams P) {
+  __shared__ float o_s[3][128];
+  const int ridx = blockIdx.x, h = blockIdx.y, lane = threadIdx.x & 31, a = threadIdx.x >> 5;
   float* w = P.rowerr + ((size_t)h * P.n_rows + ridx) * 3;
   const int r = P.rows[ridx];
-  if (r < 0 || r >= P.N) {  // rows outside the sequence contribute nothing
-    if (lane < 3) w[lane] = 0.f;
+  if (r < 0 || r >= P.N) {  // rows outside the sequence contribute nothing (the whole block leaves)
+    if (threadIdx.x < 3) w[threadIdx.x] = 0.f;
     return;
   }
-  const int D = P.D, W = D + 2;
-  const float* base = P.part + ((size_t)h * P.n_rows + ridx) * P.G * 3 * W;
-  float out[3][4];  // dims lane + 32 x, x < D / 32
+  const int D = P.D, W = D + 2, G = P.G;
+  const float* base = P.part + ((size_t)h * P.n_rows + ridx) * G * 3 * W;
+  const float* mine = base + (lane * 3 + a) * W;  // this lane's chunk, lane < G
+  const float mg = lane < G ? mine[D] : -INFINITY;
+  const float lg = lane < G ? mine[D + 1] : 0.f;
+  const float M = warp_max(mg);
+  const float fl = (mg == -INFINITY) ? 0.f : exp2f(mg - M);
+  const float L = warp_sum(lg * fl);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int g = 0; g < G; ++g) {
+    const float f = __shfl_sync(0xffffffffu, fl, g);
+    const float* src = base + (g * 3 + a) * W;
 #pragma unroll
-  for (int a = 0; a < 3; ++a) {
-    float M = -INFINITY;
-    for (int g = 0; g < P.G; ++g) M = fmaxf(M, base[(g * 3 + a) * W + D]);
-    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int g = 0; g < P.G; ++g) {
-      const float* src = base + (g * 3 + a) * W;
-      const float mg = src[D];
-      const float f = (mg == -INFINITY) ? 0.f : exp2f(mg - M);
-      L = fmaf(src[D + 1], f, L);
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-        if (lane + 32 * x < D) acc[x] = fmaf(src[lane + 32 * x], f, acc[x]);
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-    for (int x = 0; x < 4; ++x) out[a][x] = acc[x] * inv;
+    for (int x = 0; x < 4; ++x)
+      if (lane + 32 * x < D) acc[x] = fmaf(src[lane + 32 * x], f, acc[x]);
   }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+    if (lane + 32 * x < D) o_s[a][lane + 32 * x] = acc[x] * inv;
+  __syncthreads();
+  if (a != 0) return;
   float es = 0.f, et = 0.f, ed = 0.f;
 #pragma unroll
   for (int x = 0; x < 4; ++x) {
     if (lane + 32 * x >= D) continue;
-    const float od = out[0][x], os = out[1][x], ot = out[2][x];
+    const float od = o_s[0][lane + 32 * x], os = o_s[1][lane + 32 * x], ot = o_s[2][lane + 32 * x];
     es = fmaf(os - od, os - od, es);
     et = fmaf(ot - od, ot - od, et);
     ed = fmaf(od, od, ed);
@@ -549,17 +566,21 @@ __global__ void route_merge_kernel(const RouteParams P) {
   }
 }
 
-// One thread per head: fixed-order sums over the sampled rows, then the route.
+// One warp per head: fixed-order sums over the sampled rows (lane j takes rows j, j + 32, ...,
+// then a butterfly over the lanes; the order never depends on timing), then the route.
 __global__ void route_reduce_kernel(const RouteParams P) {
-  const int h = blockIdx.x * blockDim.x + threadIdx.x;
-  if (h >= P.H) return;
+  const int h = blockIdx.x, lane = threadIdx.x;
   double es = 0.0, et = 0.0, ed = 0.0;
-  for (int r = 0; r < P.n_rows; ++r) {
+  for (int r = lane; r < P.n_rows; r += 32) {
     const float* w = P.rowerr + ((size_t)h * P.n_rows + r) * 3;
     es += w[0];
     et += w[1];
     ed += w[2];
   }
+  es = warp_sum(es);
+  et = warp_sum(et);
+  ed = warp_sum(ed);
+  if (lane != 0) return;
   const double den = ed > 0.0 ? ed : 1.0;
   P.route[h] = (es <= et) ? SVG_ROUTE_SPATIAL : SVG_ROUTE_TEMPORAL;
   if (P.err) {
@@ -619,8 +640,8 @@ int launch_route(const void* q, const CUtensorMap* tm_k, const CUtensorMap* tm_v
   if (e != cudaSuccess) return record_cuda_error("cudaMemsetAsync(route status)", e);
   e = d == 128 ? launch_tc<128>(T, nblk_rows, st) : launch_tc<64>(T, nblk_rows, st);
   if (e != cudaSuccess) return record_cuda_error("launch route_tc_kernel", e);
-  route_merge_kernel<<<dim3(n_rows, heads), 32, 0, st>>>(P);
-  route_reduce_kernel<<<(heads + 127) / 128, 128, 0, st>>>(P);
+  route_merge_kernel<<<dim3(n_rows, heads), 96, 0, st>>>(P);
+  route_reduce_kernel<<<heads, 32, 0, st>>>(P);
   e = cudaGetLastError();
   return e == cudaSuccess ? SVG_OK : record_cuda_error("launch route kernels", e);
 }
