@@ -885,8 +885,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           mbar_arrive(c.s_free(h));
         }
         mask_scores<BK>(P, inf.cls, f, c0, prow, ent, lo, hi, se, per, r);
-        const bool rescale = max_first<BK>(r, sl2, m, l, alpha);
-        exp_tile<BK>(r, sl2, m, acc);
+        bool rescale = false;
+        // Exponentials against the running maximum first, without the tile's maximum: when every
+        // row's P sums to at most 2^kRescaleLog2, no P exceeds it, which is exactly when the
+        // maximum-first step would not rescale, so the result is the same bit for bit. Otherwise
+        // (rare) the tile is read again from TMEM, where S still is, and taken maximum first. With
+        // P in shared memory S may already be overwritten, so that schedule always takes the maximum.
+        bool max_step = PS || !__all_sync(0xffffffffu, m != -INFINITY);
+#pragma unroll 1
+        for (int pass = 0;; ++pass) {
+          if (max_step) {
+            if (pass > 0) {
+              load_scores<BK>(tS, r);
+              mask_scores<BK>(P, inf.cls, f, c0, prow, ent, lo, hi, se, per, r);
+            }
+            rescale = max_first<BK>(r, sl2, m, l, alpha);
+          }
+          exp_tile<BK>(r, sl2, m, acc);
+          if (max_step) break;
+          const float lt = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+          if (!__any_sync(0xffffffffu, !(lt <= kRescaleBound))) break;
+          max_step = true;
+        }
         l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
         if constexpr (PS) {
           // the previous P_h V is complete: P_h's buffer is free and O_h holds every earlier P V

@@ -627,6 +627,8 @@ __device__ __forceinline__ void exp_pack_64(uint32_t* r, float2 sc, float2 nb, f
 
 // A row maximum may grow by up to 2^kRescaleLog2 before O and l are rescaled (log2 units).
 constexpr float kRescaleLog2 = 8.0f;
+constexpr float kRescaleBound = 256.0f;  // 2^kRescaleLog2: the largest P taken without a rescale
+static_assert(kRescaleBound == (float)(1 << (int)kRescaleLog2), "rescale bound");
 
 // ---------------------------------------------------------------------------------------
 // Softmax steps of one score row (one thread per query row, BK scores in registers).
