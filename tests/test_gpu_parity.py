@@ -473,6 +473,14 @@ FUSED_CASES = [
                   spatial_band=3, sink_frames=2, bq=256, bk=64), {}),
     (syn.Workload("fused_d64_ragged", frames=5, grid_h=6, grid_w=9, routes=(1, 1, 0), d=64, frame_window=0,
                   spatial_band=2, bq=64, bk=64), {}),
+    # runs of one patch's frames longer than a tile (256 rows: boxes never fit, every group gathered),
+    # longer than a box may be (259 rows: the box maps are not built), and of a single frame
+    (syn.Workload("fused_run_256", frames=257, grid_h=2, grid_w=3, routes=(1, 0), d=128, frame_window=2,
+                  spatial_band=1), {}),
+    (syn.Workload("fused_run_259", frames=260, grid_h=2, grid_w=3, routes=(1,), d=128, frame_window=2,
+                  spatial_band=1), {}),
+    (syn.Workload("fused_run_1", frames=2, grid_h=16, grid_w=20, routes=(1, 0), d=128, frame_window=1,
+                  spatial_band=7), {}),
 ]
 
 
