@@ -1,10 +1,11 @@
 """Head-sharded attention over several GPUs (one process per GPU, torch.distributed).
 
 Heads never exchange data during the forward pass (each head attends over its own K/V under its
-own route's mask; "Sparse Attention Patterns" in the marsel.app article), so one call's heads can be
-split across ranks. Each rank then runs the attention of its heads with no collective. The only
-exchange is optional: when one device needs the whole output, `gather_heads` assembles O over the
-process group (an all-gather; NCCL over NVLink on GPUs).
+own route's mask; "Sparse Attention Patterns" in "Google Speeds Up Video Diffusion on TPUs with
+Optimized Sparse Attention"), so one call's heads can be split across ranks. Each rank then runs
+the attention of its heads with no collective. The only exchange is optional: when one device needs
+the whole output, `gather_heads` assembles O over the process group (an all-gather; NCCL over
+NVLink on GPUs).
 
 Balance: a head costs the visited half-tiles of its route's tile map (`pair_half_tiles` of the
 tile-map summary), so spatial and temporal heads weigh what they compute. Heads go to ranks
