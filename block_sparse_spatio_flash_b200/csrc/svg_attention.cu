@@ -20,7 +20,9 @@
 //  * option PS: P goes to shared memory instead, so the next tile's S is computed while the
 //    softmax of this tile runs (measured slower on B200; kept selectable);
 //  * O is rescaled (in TMEM) only when a row maximum grows by more than 2^8, which keeps
-//    the result exact while making the correction rare;
+//    the result exact while making the correction rare; after a row's first tile the
+//    exponentials are taken against the running maximum, and the tile's own maximum only when
+//    a row's P sums past 2^8 (the tile is then read again from TMEM);
 //  * every wait is bounded by a wall-clock limit; a timeout sets the status word and all
 //    roles drain their in-flight copies / MMAs and return.
 //  * fused token order: temporal heads read their tiles where the rows lie in the original order
