@@ -258,7 +258,8 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="use only the first H heads of the workload")
     ap.add_argument("--shard-heads", action="store_true",
                     help="split one call's heads over the ranks (strong scaling) instead of running replicas")
-    ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
+    ap.add_argument("--cpu-rows", type=int, default=3072,
+                    help="oracle rows per head for cpu_baseline (about 10 s of host work at the pages' shape)")
     ap.add_argument("--ref-rows", type=int, default=96, help="oracle rows per head per --impl reference step")
     ap.add_argument("--route-calls", type=int, default=0,
                     help="after the timed region, this many svg_route_heads calls (64 sampled rows per head) on the "
