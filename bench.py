@@ -366,7 +366,7 @@ def main():
     achieved = vis_flop / (statistics.mean(per_step) * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": captured_traffic(w, args),
-                "kernel": f"attn_kernel<128,128> ({args.mode}{', fused token order' if args.fused else ''}, "
+                "kernel": f"attn_kernel<{w.d},{args.bk}> ({args.mode}{', fused token order' if args.fused else ''}, "
                           f"{kernel_variant()} schedule)",
                 "flop_definition": "4*d*(in-range area of visited tiles)", "peak_kind": f"{peak_kind} bf16 burst"}
 
