@@ -7,7 +7,8 @@
   values and LSE = ln #kept; V = 1 gives O = 1; an all-kept mask gives textbook softmax
   attention computed with numpy), and a numpy brute force with an explicit N x N mask;
 * the token order against closed-form positions and the bijection property;
-* the pages' kept share (~38.87% at 75,600 tokens) for the temporal band reading.
+* the pages' kept share (~38.87% at 75,600 tokens) for the temporal band reading, and the pages'
+  38.87% and 27.55% as the spatial mask's visited and boundary tile shares at TPU tile sizes.
 """
 import math
 import os
@@ -168,6 +169,34 @@ def test_pages_shape_and_budget():
     assert sp == 152 * S * S == 1969920000
     # 1440p: four times the tokens of 720p at the same frame count
     assert syn.P1440.tokens == g["resolution_scale_tokens"] * N
+
+
+def test_pages_tile_shares_at_tpu_scale_tiles():
+    """The pages' 38.87% and 27.55% are tile-level shares of the spatial mask at TPU tile sizes.
+
+    The pages give no tile shape. Classified element by element by the oracle at 75,600 tokens
+    (+-3 frames, frame-0 sink), the share of (query tile, key tile) pairs that are visited at
+    2048 x 2048 tiles is 38.86% (the pages print 38.87% as the kept share), and the share of
+    visited tiles that are boundary tiles at 2304 x 2048 is 27.56% (the pages print 27.55%);
+    at B200's 128 x 128 tiles it is 1.7%. No single shape gives both printed values, so the
+    reading is recorded and pinned here, not used to choose the kernel's tiles; the pages'
+    2.22% after tile-aligned traversal stays unpinned (the rounded map's ragged-tail tiles are
+    3.2-3.7% of its visited tiles at these shapes)."""
+    g = read_golden("pages_workload.txt")
+    w = syn.SPATIAL_75K
+    T, S = w.frames, w.frame_size
+
+    def shares(bq, bk):
+        _, cls = oracle.tile_counts(syn.ROUTE_SPATIAL, syn.LAYOUT_SINK_PREFIX, T, S, w.frame_window, 0,
+                                    w.sink_frames, bq, bk)
+        full, bnd = int((cls == 1).sum()), int((cls == 2).sum())
+        return (full + bnd) / cls.size, bnd / (full + bnd)
+
+    visited, _ = shares(2048, 2048)
+    assert abs(visited - g["kept_pairs_percent"] / 100.0) < 2e-4
+    _, boundary = shares(2304, 2048)
+    assert abs(boundary - g["boundary_tiles_percent"] / 100.0) < 2e-4
+    assert g["boundary_tiles_aligned_percent"] < g["boundary_tiles_percent"]
 
 
 # ----------------------------------------------------------------------------- token order
